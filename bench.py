@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Throughput of Jet-Long dynamic bifocal RoPE attention on B200.
+
+One step = the whole hot path on its headline workloads:
+  * one prefill of the 128K workload (B=1, Hq=32, Hkv=8, d=128, L=131072,
+    w_pretrained=32768 so G=4, w0=4096, rope_theta=1e6, bf16), and
+  * one full pass of the decode workload (B=8, Hq=32, Hkv=8, d=128, raw-K/V
+    cache of 131136 rows, 64 single-token steps at L = 131041..131104, so G
+    goes 4 -> 5 inside the pass).
+value = prefill TFLOP/s on computed FLOPs (whole job: all ranks' FLOPs / max
+rank time).  The decode figures (GB/s of K/V streamed, tokens/s) ride along in
+"decode".  Inputs are larger than L2 (q alone is 1 GiB, the caches 4.3 GB), so
+no explicit flush is done between steps.
+
+--impl reference times the fp64 CPU oracle (the only reference this method has
+here) on a bounded sample of the same workload.
+Multi-GPU: replicas only (each rank runs the same independent workload), weak
+scaling, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from rope_context_extension_jet_b200 import inputs as I  # noqa: E402
+
+METRIC = "bifocal prefill TFLOP/s & % bf16 peak at L=128K; decode HBM GB/s"
+BM = BN = 128  # tile shape used to count computed FLOPs
+
+
+def tile_counts(L, w0, bm=BM, bn=BN):
+    """(causal tiles, band tiles) of the (query-block, key-block) grid."""
+    nqb = (L + bm - 1) // bm
+    tiles = band = 0
+    for qb in range(nqb):
+        i_lo, i_hi = qb * bm, min(qb * bm + bm - 1, L - 1)
+        nkb = i_hi // bn + 1
+        tiles += nkb
+        for kb in range(nkb):
+            j_lo, j_hi = kb * bn, kb * bn + bn - 1
+            dmax, dmin = i_hi - j_lo, max(0, i_lo - j_hi)
+            if dmin < w0 <= dmax:
+                band += 1
+    return tiles, band
+
+
+def prefill_flops(w):
+    useful = 4.0 * w.d * w.Hq * w.B * w.L * (w.L + 1) / 2
+    tiles, band = tile_counts(w.L, min(w.w0, w.L))
+    computed = w.B * w.Hq * (tiles * 4.0 * w.d * BM * BN + band * 2.0 * w.d * BM * BN)
+    return useful, computed, tiles, band
+
+
+def decode_bytes(w, L):
+    el = 2 if w.dtype == "bf16" else 4
+    kv = 2.0 * w.B * w.Hkv * L * w.d * el
+    qo = 2.0 * w.B * w.Hq * w.d * el
+    return kv, kv + qo
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def to_dev(a, dev):
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(a).to(dev)
+
+
+def to_pinned(a):
+    import torch
+    t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+    t = t.pin_memory()
+    return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+
+
+def oracle_prefill_sample(w, budget_s=20.0, nthreads=0):
+    """Time the fp64 oracle on seeded rows of the prefill workload until ~budget_s."""
+    import oracle
+    q, k, v = I.prefill_inputs(w)
+    rng = np.random.default_rng(77)
+    cores = nthreads or os.cpu_count()
+    done_rows = 0
+    flops = 0.0
+    t_total = 0.0
+    batch = max(1, cores)
+    while t_total < budget_s:
+        h = rng.integers(0, w.Hq, size=batch)
+        i = rng.integers(0, w.L, size=batch)
+        rows = np.stack([np.zeros(batch, np.int64), h, i], axis=1)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(q, k, v, rows, w0=w.w0, w_pretrained=w.w_pretrained,
+                            rope_theta=w.rope_theta, scale=w.scale, nthreads=nthreads)
+        t_total += time.perf_counter() - t0
+        done_rows += batch
+        flops += float(np.sum(4.0 * w.d * (i + 1)))
+        if t_total > 0.5 and t_total * 2 < budget_s:
+            batch *= 2
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": int(cores),
+            "kind": "oracle", "seconds": round(t_total, 2),
+            "sample": f"{done_rows} random query rows (head, position) of the 128K prefill, "
+                      f"fp64, useful FLOPs 4*d*(i+1) per row"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = I.C4
+    steps = []
+    per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for s in range(args.warmup + args.steps):
+        r = oracle_prefill_sample(w, budget_s=per)
+        if s >= args.warmup:
+            steps.append(r)
+    val = float(np.mean([r["value"] for r in steps]))
+    secs = float(np.sum([r["seconds"] for r in steps]))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1000.0 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L": w.L,
+                   "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.rope_theta},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": steps[0]["cores"],
+                         "kind": "oracle", "sample": steps[0]["sample"]},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import rope_context_extension_jet_b200 as jl
+
+    jl.load_library()  # fails loudly without the built library
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    wp, wd = I.C4, I.D
+    stream = torch.cuda.current_stream(dev)
+
+    # ---------------- inputs (host, seeded), then resident in HBM
+    q, k, v = I.prefill_inputs(wp)
+    qd, kd, vd = to_dev(q, dev), to_dev(k, dev), to_dev(v, dev)
+    outd = torch.empty_like(qd)
+    dq, dkc, dvc = I.decode_inputs(wd)
+    dqd, dkcd, dvcd = to_dev(dq, dev), to_dev(dkc, dev), to_dev(dvc, dev)
+    del dkc, dvc
+    dout = torch.empty_like(dqd[0])
+    ws = torch.empty(jl.decode_workspace_size(wd.B, wd.Hq, wd.Hkv, wd.Lcap, wd.d),
+                     dtype=torch.uint8, device=dev)
+
+    def prefill_call():
+        jl.prefill(qd, kd, vd, outd, w0=wp.w0, w_pretrained=wp.w_pretrained,
+                   rope_theta=wp.rope_theta, scale=wp.scale, stream=stream)
+
+    def decode_call(t):
+        jl.decode(dqd[t], dkcd, dvcd, wd.length_at(t), dout, w0=wd.w0,
+                  w_pretrained=wd.w_pretrained, rope_theta=wd.rope_theta, scale=wd.scale,
+                  workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill_call()
+        for t in range(wd.steps):
+            decode_call(t)
+    jl.device_status(stream)
+
+    # ---------------- timed region (device time, CUDA events on the launching stream)
+    sampler = ClockSampler(local)
+    ev_p = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = jl.launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev_p[s][0].record(stream)
+        prefill_call()
+        ev_p[s][1].record(stream)
+        ev_d[s][0].record(stream)
+        for t in range(wd.steps):
+            decode_call(t)
+        ev_d[s][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = jl.launch_count() - launches0
+    barrier()
+    clocks = sampler.stop()
+    jl.device_status(stream)
+
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    pre_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev_p])))
+    dec_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev_d])))
+
+    useful, computed, tiles, band = prefill_flops(wp)
+    pre_tflops = world * computed / (pre_ms * 1e-3) / 1e12
+    pre_useful_tflops = world * useful / (pre_ms * 1e-3) / 1e12
+    kv_bytes = sum(decode_bytes(wd, wd.length_at(t))[0] for t in range(wd.steps))
+    all_bytes = sum(decode_bytes(wd, wd.length_at(t))[1] for t in range(wd.steps))
+    dec_gbs = world * kv_bytes / (dec_ms * 1e-3) / 1e9
+    dec_tok_s = world * wd.B * wd.steps / (dec_ms * 1e-3)
+
+    # ---------------- end to end through the public API with host buffers
+    qh, kh, vh = to_pinned(q), to_pinned(k), to_pinned(v)
+    outh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
+    e2e_ev = []
+    for s in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        prefill_call()
+        outh.copy_(outd, non_blocking=True)
+        b.record(stream)
+        if s >= args.warmup:
+            e2e_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])))
+    h2d = sum(x.numel() * x.element_size() for x in (qd, kd, vd))
+    d2h = outd.numel() * outd.element_size()
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = oracle_prefill_sample(wp, budget_s=args.cpu_budget)
+        frac_s = pre_tflops / world / peaks["bf16_tflops_sustained"]
+        line = {
+            "metric": METRIC, "value": round(pre_tflops, 2), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) q/k/v, bf16)",
+            "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d,
+                       "L": wp.L, "w_pretrained": wp.w_pretrained, "G": jl.group_size(wp.L, wp.w_pretrained),
+                       "w0": wp.w0, "rope_theta": wp.rope_theta,
+                       "decode_workload": wd.name, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "prefill": {"ms": round(pre_ms, 3), "tflops_computed": round(pre_tflops, 2),
+                        "tflops_useful": round(pre_useful_tflops, 2),
+                        "flops_computed": computed, "flops_useful": useful,
+                        "tiles": tiles, "band_tiles": band,
+                        "tokens_per_s": round(world * wp.B * wp.L / (pre_ms * 1e-3), 1),
+                        "frac_of_sustained_bf16": round(frac_s, 4),
+                        "frac_of_burst_bf16": round(pre_tflops / world / peaks["bf16_tflops"], 4)},
+            "decode": {"ms_per_token_step": round(dec_ms / wd.steps, 4),
+                       "gbs_kv": round(dec_gbs, 1), "bytes_per_pass_kv": kv_bytes,
+                       "bytes_per_pass_all": all_bytes, "tokens_per_s": round(dec_tok_s, 1),
+                       "frac_of_hbm": round(dec_gbs / world / peaks["hbm_gbs"], 4),
+                       "G": [jl.group_size(wd.length_at(0), wd.w_pretrained),
+                             jl.group_size(wd.length_at(wd.steps - 1), wd.w_pretrained)]},
+            "roofline": {"bound": "tensor", "achieved": round(pre_tflops / world, 2),
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": round(frac_s, 4), "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 sustained"},
+            "e2e": {"value": round(world * computed / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,117 @@
+/*
+ * jetlong.h -- C ABI of libjetlong: Jet-Long dynamic bifocal RoPE causal
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * Method ("Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
+ * RoPE", gist.science/it/paper/2607.07740):
+ *   - Metodologia 1 "RoPE Bifocale Dinamico": for a query at position i and a
+ *     key at position j, pairs closer than a local window w0 (i - j < w0) use
+ *     classic RoPE at the exact positions i and j; all other pairs use RoPE at
+ *     the aliased positions f(i), f(j) with f(x) = floor(x / G) and
+ *     G = max(1, ceil(L / w_pretrained)) recomputed from the current length L.
+ *   - Metodologia 2 "Meccanismi di Efficienza dell'Inferenza": the KV cache
+ *     keeps unrotated base keys and is never rewritten; the rotations are
+ *     applied on the fly (rotations compose additively); both branches feed one
+ *     exact softmax (the pages reach it by an inclusion-exclusion merge of three
+ *     attention passes; this library computes the same routed result in one
+ *     fused pass with a per-element branch select on boundary tiles).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are contiguous row-major.  Prefill: q, out [B, Hq, L, d];
+ *     k, v [B, Hkv, L, d].  Decode: q, out [B, Hq, d]; kcache, vcache
+ *     [B, Hkv, Lcap, d] with rows [0, L) valid.
+ *   - q, k and the caches hold UNROTATED ("raw") vectors: the library applies
+ *     every rotation.  Frequencies theta_m = rope_theta^(-2m/d), m < d/2,
+ *     half-split pairing (x_m, x_{m+d/2}).  Grouped-query attention: q head h
+ *     reads kv head h / (Hq / Hkv).  Softmax is softmax(scale * logit), base e.
+ *   - Element type: JETLONG_BF16 (q, k, v, caches and out are bf16; tensor-core
+ *     path for prefill) or JETLONG_FP32 (all fp32; CUDA-core fp32 path).
+ *     Accumulation is fp32 in both.
+ *   - All pointers named d_* or tensor pointers are DEVICE memory owned by the
+ *     caller.  The library never writes q, k, v or the caches and allocates no
+ *     device memory in any call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) on the current device.
+ *   - Errors: every entry point returning int returns a jetlong_status.
+ *     Arguments are validated on the host before any launch; on failure nothing
+ *     is launched and jetlong_last_error() describes the problem.
+ */
+#ifndef JETLONG_H
+#define JETLONG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { JETLONG_BF16 = 0, JETLONG_FP32 = 1 } jetlong_dtype;
+
+typedef enum {
+    JETLONG_OK = 0,
+    JETLONG_ERR_INVALID_ARG = 1, /* bad pointer, size or parameter          */
+    JETLONG_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d)      */
+    JETLONG_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed    */
+    JETLONG_ERR_TIMEOUT = 4      /* a bounded device wait gave up           */
+} jetlong_status;
+
+/* Dynamic group size G = max(1, ceil(L / w_pretrained)) (Metodologia 1,
+ * display equation).  Pure host function, int64 arithmetic.  Returns -1 if
+ * L < 0 or w_pretrained < 1. */
+int64_t jetlong_group_size(int64_t L, int64_t w_pretrained);
+
+/* Aliased position map of Metodologia 1: d_out[x] = floor(x / G) for
+ * x in [0, L), G = jetlong_group_size(L, w_pretrained).  d_out: device int32
+ * array of L elements.  L must be in [1, 2^31 - 1].  Asynchronous on stream. */
+int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* stream);
+
+/* Prefill: routed causal attention of every query row of a length-L sequence
+ * against keys [0, i] with one G for the call (from this L).
+ *   q [B,Hq,L,d], k/v [B,Hkv,L,d] raw inputs; out [B,Hq,L,d] written.
+ *   w0 >= 0 local window (w0 = 0: every pair remote; w0 >= L: every pair local);
+ *   w_pretrained >= 1; rope_theta > 1; scale > 0 and finite.
+ *   d must be 64 or 128 (else JETLONG_ERR_UNSUPPORTED); Hq % Hkv == 0.
+ * Sizes: B*Hq*L*d < 2^31 per tensor is NOT required; L < 2^31. */
+int jetlong_prefill(const void* q, const void* k, const void* v, void* out,
+                    int B, int Hq, int Hkv, int L, int d,
+                    int w0, int w_pretrained, double rope_theta, float scale,
+                    jetlong_dtype dtype, void* stream);
+
+/* Bytes of device workspace jetlong_decode needs for any L <= Lcap with these
+ * sizes (partial softmax states of the key splits plus merge counters).
+ * Returns 0 for invalid sizes. */
+size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int Lcap, int d);
+
+/* Decode: one new query per (b, h) at position i = L - 1 attending cache rows
+ * [0, L), with G recomputed from this L (so G changes as generation crosses a
+ * multiple of w_pretrained while the cache is untouched, Metodologia 2).  The
+ * caller appends the new token's raw key/value at row L - 1 beforehand.
+ *   q [B,Hq,d] raw, kcache/vcache [B,Hkv,Lcap,d] raw, out [B,Hq,d] written.
+ *   1 <= L <= Lcap.  workspace: device memory of at least
+ *   jetlong_decode_workspace_size(B,Hq,Hkv,Lcap,d) bytes, 16-byte aligned,
+ *   owned by the caller; its contents on entry do not matter.  Two calls that
+ *   share one workspace must not overlap on the device. */
+int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* out,
+                   int B, int Hq, int Hkv, int L, int Lcap, int d,
+                   int w0, int w_pretrained, double rope_theta, float scale,
+                   jetlong_dtype dtype, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/* Synchronises `stream`, then reads and clears the library's device error
+ * word, set by a kernel whose bounded wait expired (the kernel then returned
+ * without finishing its tile).  Returns JETLONG_OK, JETLONG_ERR_TIMEOUT or
+ * JETLONG_ERR_CUDA. */
+int jetlong_device_status(void* stream);
+
+/* Message for the last failing call on this host thread ("" if none). */
+const char* jetlong_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t jetlong_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JETLONG_H */

@@ -1,0 +1,183 @@
+"""Jet-Long dynamic bifocal RoPE attention for NVIDIA B200 -- Python binding.
+
+Thin ctypes binding of ``libjetlong.so`` (C ABI declared in ``include/jetlong.h``).
+Functions keep the C names without the ``jetlong_`` prefix.  This module only
+marshals arguments: torch tensors supply device pointers and the current CUDA
+stream; every step of the attention runs in the library's CUDA kernels.  There
+is no fallback: if the library is missing the calls raise.
+
+Method: "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
+(gist.science/it/paper/2607.07740), Metodologia 1 (local window w0 with classic
+RoPE; remote pairs at f(x) = floor(x/G), G = max(1, ceil(L/w_pretrained))) and
+Metodologia 2 (rotations applied on the fly to an untouched cache; one exact
+distance-routed softmax).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "BF16", "FP32", "JetLongError", "load_library", "group_size", "position_map", "prefill",
+    "decode_workspace_size", "decode", "device_status", "last_error", "launch_count",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libjetlong.so")
+
+BF16 = 0
+FP32 = 1
+_STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class JetLongError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"jetlong {_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def load_library(path: str | None = None):
+    """Load libjetlong.so (built in-tree by ``python -m rope_context_extension_jet_b200._build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with "
+                               "`python -m rope_context_extension_jet_b200._build`")
+        lib = ctypes.CDLL(p)
+        vp, i32, i64, sz, dbl, flt = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_size_t, ctypes.c_double, ctypes.c_float)
+        lib.jetlong_group_size.restype = i64
+        lib.jetlong_group_size.argtypes = [i64, i64]
+        lib.jetlong_position_map.restype = i32
+        lib.jetlong_position_map.argtypes = [vp, i64, i64, vp]
+        lib.jetlong_prefill.restype = i32
+        lib.jetlong_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                        dbl, flt, i32, vp]
+        lib.jetlong_decode_workspace_size.restype = sz
+        lib.jetlong_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        lib.jetlong_decode.restype = i32
+        lib.jetlong_decode.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                       dbl, flt, i32, vp, sz, vp]
+        lib.jetlong_device_status.restype = i32
+        lib.jetlong_device_status.argtypes = [vp]
+        lib.jetlong_last_error.restype = ctypes.c_char_p
+        lib.jetlong_last_error.argtypes = []
+        lib.jetlong_launch_count.restype = ctypes.c_uint64
+        lib.jetlong_launch_count.argtypes = []
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _check(status: int, lib=None):
+    if status != 0:
+        lib = lib or load_library()
+        raise JetLongError(status, lib.jetlong_last_error().decode())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _dev(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def last_error() -> str:
+    return load_library().jetlong_last_error().decode()
+
+
+def launch_count() -> int:
+    return int(load_library().jetlong_launch_count())
+
+
+def group_size(L: int, w_pretrained: int) -> int:
+    """G = max(1, ceil(L / w_pretrained)); -1 for invalid arguments."""
+    return int(load_library().jetlong_group_size(int(L), int(w_pretrained)))
+
+
+def position_map(out, L: int, w_pretrained: int, stream=None):
+    """Write floor(x / G) for x in [0, L) into the int32 CUDA tensor ``out``."""
+    import torch
+    if out.dtype != torch.int32 or out.numel() < L:
+        raise ValueError("out must be an int32 tensor with at least L elements")
+    lib = load_library()
+    _check(lib.jetlong_position_map(_dev(out, "out"), int(L), int(w_pretrained), _stream(stream)),
+           lib)
+    return out
+
+
+def prefill(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: float,
+            scale: float | None = None, stream=None):
+    """Routed causal attention over raw q [B,Hq,L,d], k/v [B,Hkv,L,d] (bf16 or fp32)."""
+    import torch
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, L, d] matching q")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_prefill(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                               B, Hq, Hkv, L, d, int(w0), int(w_pretrained), float(rope_theta),
+                               float(scale), _dtype_code(q), _stream(stream)), lib)
+    return out
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, Lcap: int, d: int) -> int:
+    return int(load_library().jetlong_decode_workspace_size(B, Hq, Hkv, Lcap, d))
+
+
+def decode(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
+           rope_theta: float, scale: float | None = None, workspace=None, stream=None):
+    """One decode step: raw q [B,Hq,d] at position L-1 over cache rows [0, L)."""
+    import torch
+    B, Hq, d = q.shape
+    _, Hkv, Lcap, _ = kcache.shape
+    if vcache.shape != kcache.shape:
+        raise ValueError("kcache and vcache must have the same shape")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_size(B, Hq, Hkv, Lcap, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_decode(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
+                              _dev(out, "out"), B, Hq, Hkv, int(L), Lcap, d, int(w0),
+                              int(w_pretrained), float(rope_theta), float(scale),
+                              _dtype_code(q), _dev(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(), _stream(stream)), lib)
+    return out
+
+
+def device_status(stream=None):
+    """Synchronise the stream and raise if a kernel's bounded wait expired."""
+    lib = load_library()
+    _check(lib.jetlong_device_status(_stream(stream)), lib)

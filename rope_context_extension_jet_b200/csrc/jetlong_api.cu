@@ -1,0 +1,224 @@
+// jetlong_api.cu -- the C ABI of libjetlong: argument validation, the dynamic
+// group size, RoPE phase constants, error state and dispatch to the kernels.
+//
+// "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
+// (gist.science/it/paper/2607.07740), Metodologia 1: G = max(1,
+// ceil(L / w_pretrained)) from the current length; f(x) = floor(x / G).
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "jl_common.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+__device__ int g_dev_error;  // set by kernels whose bounded waits expire
+
+int fail(int code, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int ok()
+{
+    g_last_error.clear();
+    return JETLONG_OK;
+}
+
+int* dev_error_word(cudaError_t* err)
+{
+    static std::mutex mu;
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_dev_error);
+        if (*err != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int Hq, int Hkv, int d, int w0, int w_pretrained, double rope_theta,
+                 float scale, jetlong_dtype dtype)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1)
+        return fail(JETLONG_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d d=%d)", B,
+                    Hq, Hkv, d);
+    if (Hq % Hkv != 0)
+        return fail(JETLONG_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (w0 < 0) return fail(JETLONG_ERR_INVALID_ARG, "w0 must be >= 0 (got %d)", w0);
+    if (w_pretrained < 1)
+        return fail(JETLONG_ERR_INVALID_ARG, "w_pretrained must be >= 1 (got %d)", w_pretrained);
+    if (!(rope_theta > 1.0) || !std::isfinite(rope_theta))
+        return fail(JETLONG_ERR_INVALID_ARG, "rope_theta must be finite and > 1");
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return fail(JETLONG_ERR_INVALID_ARG, "scale must be finite and > 0");
+    if (dtype != JETLONG_BF16 && dtype != JETLONG_FP32)
+        return fail(JETLONG_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (d != 64 && d != 128)
+        return fail(JETLONG_ERR_UNSUPPORTED, "head dim d=%d not supported (64 or 128)", d);
+    if (Hq > 65535 || B > 65535)
+        return fail(JETLONG_ERR_UNSUPPORTED, "B and Hq must be <= 65535");
+    return JETLONG_OK;
+}
+
+}  // namespace
+
+namespace jl {
+
+// omega_m = theta_m / (2 pi) as a 0.64 fixed-point turn fraction (theta_m <= 1,
+// so omega_m < 1/(2 pi)); the scaling by 2^64 is done in long double.
+void make_rope_turns(RopeTurns* t, int d, double rope_theta)
+{
+    const long double two_pi = 6.283185307179586476925286766559L;
+    memset(t, 0, sizeof *t);
+    for (int m = 0; m < d / 2; ++m) {
+        const double theta_m = std::pow(rope_theta, -2.0 * (double)m / (double)d);
+        const long double w = ((long double)theta_m / two_pi) * 18446744073709551616.0L;
+        const uint64_t W = (uint64_t)w;
+        t->hi[m] = (uint32_t)(W >> 32);
+        t->lo[m] = (uint32_t)W;
+    }
+}
+
+}  // namespace jl
+
+extern "C" {
+
+int64_t jetlong_group_size(int64_t L, int64_t w_pretrained)
+{
+    if (L < 0 || w_pretrained < 1) return -1;
+    int64_t g = L / w_pretrained + (L % w_pretrained != 0 ? 1 : 0);
+    return g < 1 ? 1 : g;
+}
+
+const char* jetlong_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t jetlong_launch_count(void) { return g_launches.load(); }
+
+int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* stream)
+{
+    if (!d_out) return fail(JETLONG_ERR_INVALID_ARG, "d_out is null");
+    if (L < 1 || L > 2147483647LL) return fail(JETLONG_ERR_INVALID_ARG, "L out of range");
+    if (w_pretrained < 1) return fail(JETLONG_ERR_INVALID_ARG, "w_pretrained must be >= 1");
+    const int64_t G = jetlong_group_size(L, w_pretrained);
+    int n = 0;
+    cudaError_t e = jl::launch_position_map(d_out, (int)L, (int)G, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "position map launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                    int Hkv, int L, int d, int w0, int w_pretrained, double rope_theta,
+                    float scale, jetlong_dtype dtype, void* stream)
+{
+    if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(JETLONG_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (L < 1) return fail(JETLONG_ERR_INVALID_ARG, "L must be >= 1 (got %d)", L);
+    int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
+    if (st != JETLONG_OK) return st;
+    cudaError_t e;
+    int* derr = dev_error_word(&e);
+    if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+
+    jl::PrefillProblem p{};
+    p.q = q; p.k = k; p.v = v; p.out = out;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.d = d;
+    p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
+    p.G = (int)jetlong_group_size(L, w_pretrained);
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    jl::make_rope_turns(&p.turns, d, rope_theta);
+    p.dev_error = derr;
+    int n = 0;
+    e = jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int Lcap, int d)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Lcap < 1 || d < 1 || Hq % Hkv) return 0;
+    if (d != 64 && d != 128) return 0;
+    return jl::decode_workspace_bytes(B, Hq, Hkv, Lcap, d);
+}
+
+int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* out, int B,
+                   int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                   double rope_theta, float scale, jetlong_dtype dtype, void* workspace,
+                   size_t workspace_bytes, void* stream)
+{
+    if (!q || !kcache || !vcache || !out || !workspace)
+        return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
+        !aligned16(workspace))
+        return fail(JETLONG_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if (L < 1 || Lcap < L)
+        return fail(JETLONG_ERR_INVALID_ARG, "need 1 <= L <= Lcap (L=%d Lcap=%d)", L, Lcap);
+    int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
+    if (st != JETLONG_OK) return st;
+    if ((int64_t)B * Hkv > 65535 * 64)
+        return fail(JETLONG_ERR_UNSUPPORTED, "B * Hkv too large");
+    const size_t need = jl::decode_workspace_bytes(B, Hq, Hkv, Lcap, d);
+    if (workspace_bytes < need)
+        return fail(JETLONG_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)",
+                    workspace_bytes, need);
+    cudaError_t e;
+    int* derr = dev_error_word(&e);
+    if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+
+    jl::DecodeProblem p{};
+    p.q = q; p.kc = kcache; p.vc = vcache; p.out = out;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.Lcap = Lcap; p.d = d;
+    p.w0 = w0 > L ? L : w0;
+    p.G = (int)jetlong_group_size(L, w_pretrained);
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    jl::make_rope_turns(&p.turns, d, rope_theta);
+    p.workspace = workspace;
+    p.workspace_bytes = workspace_bytes;
+    p.dev_error = derr;
+    int n = 0;
+    e = jl::launch_decode(p, dtype, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int jetlong_device_status(void* stream)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+    int* derr = dev_error_word(&e);
+    if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+    int h = 0;
+    e = cudaMemcpy(&h, derr, sizeof h, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+    if (h != 0) {
+        int z = 0;
+        cudaMemcpy(derr, &z, sizeof z, cudaMemcpyHostToDevice);
+        return fail(JETLONG_ERR_TIMEOUT, "a bounded device wait expired (code 0x%x)", h);
+    }
+    return ok();
+}
+
+}  // extern "C"

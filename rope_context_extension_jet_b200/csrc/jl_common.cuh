@@ -1,0 +1,112 @@
+// jl_common.cuh -- declarations shared by the libjetlong translation units.
+//
+// RoPE phase arithmetic.  The rotation angle of pair m at position p is
+// p * theta_m with theta_m = rope_theta^(-2m/d) (standard RoPE frequencies,
+// half-split pairing; the pages evaluate Qwen3 models, which use this form).
+// Positions reach 131071 and theta_0 = 1 rad/token, so the plain fp32 product
+// p * theta_m would be off by ~1e-2 rad.  Instead the host stores
+// omega_m = theta_m / (2 pi) as an unsigned 0.64 fixed-point fraction of a
+// turn; the device forms the angle's fractional turn exactly as the low 64 bits
+// of p * omega_m (only the top 32 are needed), converts that to an fp32 value
+// in [-0.5, 0.5) and calls CUDA's sincospif / __sincosf on it.  The resulting
+// angle error is ~1e-7 rad at any position (rounding of the fp32 turn value).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "jetlong.h"
+
+namespace jl {
+
+constexpr int kMaxHalf = 64;  // d <= 128
+
+// omega_m = theta_m / (2 pi) in 0.64 fixed point, split into 32-bit words.
+struct RopeTurns {
+    uint32_t hi[kMaxHalf];
+    uint32_t lo[kMaxHalf];
+};
+
+void make_rope_turns(RopeTurns* t, int d, double rope_theta);
+
+// Fractional turn of p * omega (exact modulo 2^-32 turn), as fp32 in [-0.5, 0.5).
+__device__ __forceinline__ float rope_turn(uint32_t p, uint32_t w_hi, uint32_t w_lo)
+{
+    uint32_t top = p * w_hi + __umulhi(p, w_lo);
+    return (float)(int32_t)top * 2.3283064365386963e-10f;  // 2^-32
+}
+
+// Accurate cos/sin of the angle of pair m at position p (sincospif, ~1 ulp).
+__device__ __forceinline__ void rope_cs_accurate(uint32_t p, uint32_t w_hi, uint32_t w_lo,
+                                                 float& c, float& s)
+{
+    float t = rope_turn(p, w_hi, w_lo);
+    sincospif(2.0f * t, &s, &c);
+}
+
+// Fast cos/sin (hardware approximations on the reduced angle in [-pi, pi);
+// absolute error ~5e-7).
+__device__ __forceinline__ void rope_cs_fast(uint32_t p, uint32_t w_hi, uint32_t w_lo,
+                                             float& c, float& s)
+{
+    float t = rope_turn(p, w_hi, w_lo);
+    __sincosf(6.28318530717958647692f * t, &s, &c);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+template <typename T> __device__ __forceinline__ float load_elem(const T* p);
+template <> __device__ __forceinline__ float load_elem<float>(const float* p) { return *p; }
+template <> __device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p)
+{
+    return __bfloat162float(*p);
+}
+template <typename T> __device__ __forceinline__ void store_elem(T* p, float x);
+template <> __device__ __forceinline__ void store_elem<float>(float* p, float x) { *p = x; }
+template <> __device__ __forceinline__ void store_elem<__nv_bfloat16>(__nv_bfloat16* p, float x)
+{
+    *p = __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch plumbing shared by the translation units.
+
+struct PrefillProblem {
+    const void *q, *k, *v;
+    void* out;
+    int B, Hq, Hkv, L, d, w0;
+    int G;             // dynamic group size for this call (fits int: G <= L)
+    float scale_log2;  // scale * log2(e): logits kept in base-2 units
+    RopeTurns turns;
+    int* dev_error;    // device error word (bounded waits)
+};
+
+struct DecodeProblem {
+    const void *q, *kc, *vc;
+    void* out;
+    int B, Hq, Hkv, L, Lcap, d, w0;
+    int G;
+    float scale_log2;
+    RopeTurns turns;
+    void* workspace;
+    size_t workspace_bytes;
+    int* dev_error;
+};
+
+// Returns cudaSuccess or the launch error; each adds its launches to *nlaunch.
+cudaError_t launch_prefill_simt(const PrefillProblem& p, jetlong_dtype dt, cudaStream_t s,
+                                int* nlaunch);
+cudaError_t launch_prefill_tc(const PrefillProblem& p, cudaStream_t s, int* nlaunch);
+cudaError_t launch_decode(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s, int* nlaunch);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d);
+cudaError_t launch_position_map(int32_t* out, int L, int G, cudaStream_t s, int* nlaunch);
+
+}  // namespace jl

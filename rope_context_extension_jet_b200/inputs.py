@@ -10,16 +10,19 @@ Workload shapes follow the pages' setting (Qwen3-style grouped-query attention,
 head dim 128, a 32K native window extended to 128K): "Jet-Long: Efficient
 Long-Context Extension with Dynamic Bifocal RoPE", Risultati Sperimentali.
 
-Recipe (per workload with index n):
-  q ~ N(0,1) from default_rng(1000 + n), drawn per (b, h) as an [L, d] block;
-  k ~ N(0,1) from default_rng(2000 + n), per (b, kv-head);
-  v ~ N(0,1) from default_rng(3000 + n), per (b, kv-head);
-  outlier keys: default_rng(4000); per (b, kv-head) a permutation of [0, L),
-  its first floor(0.01 L) rows multiplied by 8 before rounding.
+Recipe (workload index n; block c = b * heads + h, one [L, d] block per head):
+  q ~ N(0,1): block c drawn by default_rng([1000 + n, c]).standard_normal(float32);
+  k ~ N(0,1): default_rng([2000 + n, c]) per (b, kv-head);
+  v ~ N(0,1): default_rng([3000 + n, c]) per (b, kv-head);
+  outlier keys: default_rng([4000, c]).permutation(L)[:floor(0.01 L)] are the rows
+  of kv block c multiplied by 8 before rounding.
+Blocks are independent streams, so they are drawn in parallel threads.
 """
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
 import numpy as np
@@ -102,41 +105,44 @@ D = DecodeWorkload("decode-bf16-B8-L131041..131104-G4to5", 4, "bf16", 8, 32, 8, 
 WORKLOADS = {"PR1": PR1, "C2": C2, "C3": C3, "C4": C4, "D": D}
 
 
-def _normal_blocks(seed: int, nblocks: int, shape) -> np.ndarray:
-    rng = np.random.default_rng(seed)
-    out = np.empty((nblocks,) + tuple(shape), dtype=np.float32)
-    for n in range(nblocks):
-        out[n] = rng.standard_normal(shape, dtype=np.float32)
+def _blocks(seed: int, nblocks: int, shape, dtype: str, transform=None) -> np.ndarray:
+    """nblocks independent N(0,1) blocks (block c from default_rng([seed, c])),
+    optionally transformed per block, then rounded to bf16 bits or kept fp32."""
+    out = np.empty((nblocks,) + tuple(shape), dtype=np.uint16 if dtype == "bf16" else np.float32)
+
+    def one(c):
+        x = np.random.default_rng([seed, c]).standard_normal(shape, dtype=np.float32)
+        if transform is not None:
+            transform(c, x)
+        out[c] = to_bf16_bits(x) if dtype == "bf16" else x
+
+    with ThreadPoolExecutor(max_workers=min(16, max(1, os.cpu_count() or 1))) as ex:
+        list(ex.map(one, range(nblocks)))
     return out
-
-
-def _finish(x: np.ndarray, dtype: str) -> np.ndarray:
-    return to_bf16_bits(x) if dtype == "bf16" else np.ascontiguousarray(x, dtype=np.float32)
 
 
 def outlier_rows(w: PrefillWorkload) -> np.ndarray:
     """Boolean [B, Hkv, L] mask of the key rows scaled for the outlier workload."""
-    mask = np.zeros((w.B, w.Hkv, w.L), dtype=bool)
+    mask = np.zeros((w.B * w.Hkv, w.L), dtype=bool)
     n_out = int(math.floor(w.outlier_frac * w.L))
-    if n_out == 0:
-        return mask
-    rng = np.random.default_rng(4000)
-    for b in range(w.B):
-        for h in range(w.Hkv):
-            mask[b, h, rng.permutation(w.L)[:n_out]] = True
-    return mask
+    if n_out:
+        for c in range(w.B * w.Hkv):
+            mask[c, np.random.default_rng([4000, c]).permutation(w.L)[:n_out]] = True
+    return mask.reshape(w.B, w.Hkv, w.L)
 
 
 def prefill_inputs(w: PrefillWorkload):
     """(q, k, v): q [B,Hq,L,d], k/v [B,Hkv,L,d]; uint16 bf16 bits or float32."""
-    q = _normal_blocks(1000 + w.index, w.B * w.Hq, (w.L, w.d)).reshape(w.B, w.Hq, w.L, w.d)
-    q = _finish(q, w.dtype)
-    k = _normal_blocks(2000 + w.index, w.B * w.Hkv, (w.L, w.d)).reshape(w.B, w.Hkv, w.L, w.d)
+    q = _blocks(1000 + w.index, w.B * w.Hq, (w.L, w.d), w.dtype).reshape(w.B, w.Hq, w.L, w.d)
+    transform = None
     if w.outlier_frac > 0:
-        k[outlier_rows(w)] *= np.float32(w.outlier_scale)
-    k = _finish(k, w.dtype)
-    v = _finish(_normal_blocks(3000 + w.index, w.B * w.Hkv, (w.L, w.d))
-                .reshape(w.B, w.Hkv, w.L, w.d), w.dtype)
+        mask = outlier_rows(w).reshape(w.B * w.Hkv, w.L)
+
+        def transform(c, x):
+            x[mask[c]] *= np.float32(w.outlier_scale)
+    k = _blocks(2000 + w.index, w.B * w.Hkv, (w.L, w.d), w.dtype, transform)
+    k = k.reshape(w.B, w.Hkv, w.L, w.d)
+    v = _blocks(3000 + w.index, w.B * w.Hkv, (w.L, w.d), w.dtype).reshape(w.B, w.Hkv, w.L, w.d)
     return q, k, v
 
 
@@ -146,12 +152,9 @@ def decode_inputs(w: DecodeWorkload):
     Rows [0, L0) are the cache before the first step; row L0 + t holds the raw
     key/value of the token appended at step t (the caller's append).
     """
-    q = _normal_blocks(1000 + w.index, w.steps, (w.B, w.Hq, w.d))
-    q = _finish(q, w.dtype)
-    kc = _finish(_normal_blocks(2000 + w.index, w.B * w.Hkv, (w.Lcap, w.d))
-                 .reshape(w.B, w.Hkv, w.Lcap, w.d), w.dtype)
-    vc = _finish(_normal_blocks(3000 + w.index, w.B * w.Hkv, (w.Lcap, w.d))
-                 .reshape(w.B, w.Hkv, w.Lcap, w.d), w.dtype)
+    q = _blocks(1000 + w.index, w.steps, (w.B, w.Hq, w.d), w.dtype)
+    kc = _blocks(2000 + w.index, w.B * w.Hkv, (w.Lcap, w.d), w.dtype).reshape(w.B, w.Hkv, w.Lcap, w.d)
+    vc = _blocks(3000 + w.index, w.B * w.Hkv, (w.Lcap, w.d), w.dtype).reshape(w.B, w.Hkv, w.Lcap, w.d)
     return q, kc, vc
 
 
