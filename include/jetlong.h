@@ -98,6 +98,31 @@ int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* 
                    jetlong_dtype dtype, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/* Allocation-free decode.  The paper has no counterpart to this entry point:
+ * it exists for callers that cannot allocate device memory at all (a serving
+ * runtime whose caching allocator must not grow, code running in a host
+ * callback, or a host framework that hands this library only the step's
+ * tensors), so they cannot supply jetlong_decode's workspace.
+ *
+ * Same arguments, semantics and results as jetlong_decode without the
+ * workspace: the split partials and merge counters live in one fixed device
+ * array of JETLONG_DECODE_NOALLOC_SCRATCH_BYTES inside the library, which every
+ * GPU that loads the library holds until the process exits.  The call allocates
+ * nothing (no cudaMalloc, no allocating library routine).
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Problems whose scratch exceeds the array are rejected with
+ *     JETLONG_ERR_INVALID_ARG before any launch (the message gives the bytes
+ *     needed); use jetlong_decode with a workspace for them.
+ *   - All calls on a device share the array and leave their contents in it.
+ *     Calls that overlap on the GPU (e.g. on two streams without ordering
+ *     between them) race on the array and give wrong results: serialise them. */
+#define JETLONG_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* out,
+                           int B, int Hq, int Hkv, int L, int Lcap, int d,
+                           int w0, int w_pretrained, double rope_theta, float scale,
+                           jetlong_dtype dtype, void* stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word, set by a kernel whose bounded wait expired (the kernel then returned
  * without finishing its tile).  Returns JETLONG_OK, JETLONG_ERR_TIMEOUT or

@@ -21,7 +21,8 @@ import threading
 
 __all__ = [
     "BF16", "FP32", "JetLongError", "load_library", "group_size", "position_map", "prefill",
-    "decode_workspace_size", "decode", "device_status", "last_error", "launch_count",
+    "decode_workspace_size", "decode", "decode_noalloc", "device_status", "last_error",
+    "launch_count", "DECODE_NOALLOC_SCRATCH_BYTES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -66,6 +67,9 @@ def load_library(path: str | None = None):
         lib.jetlong_decode.restype = i32
         lib.jetlong_decode.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                        dbl, flt, i32, vp, sz, vp]
+        lib.jetlong_decode_noalloc.restype = i32
+        lib.jetlong_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                               i32, dbl, flt, i32, vp]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -174,6 +178,36 @@ def decode(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
                               int(w_pretrained), float(rope_theta), float(scale),
                               _dtype_code(q), _dev(workspace, "workspace"),
                               workspace.numel() * workspace.element_size(), _stream(stream)), lib)
+    return out
+
+
+# Size of the library's fixed decode scratch array (JETLONG_DECODE_NOALLOC_SCRATCH_BYTES).
+DECODE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def decode_noalloc(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
+                   rope_theta: float, scale: float | None = None, stream=None):
+    """Decode step for callers that cannot allocate device memory.
+
+    Same result as ``decode`` but without a workspace: the library keeps the
+    split partials in its own fixed device array (shared by all calls on a
+    device, so calls that overlap on the GPU race).  ``out`` should be
+    preallocated by such callers; problems too large for the array raise
+    JetLongError(INVALID_ARG).
+    """
+    import torch
+    B, Hq, d = q.shape
+    _, Hkv, Lcap, _ = kcache.shape
+    if vcache.shape != kcache.shape:
+        raise ValueError("kcache and vcache must have the same shape")
+    if out is None:
+        out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_decode_noalloc(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
+                                      _dev(out, "out"), B, Hq, Hkv, int(L), Lcap, d, int(w0),
+                                      int(w_pretrained), float(rope_theta), float(scale),
+                                      _dtype_code(q), _stream(stream)), lib)
     return out
 
 

@@ -17,6 +17,8 @@
 // the last CTA of a (b, kv head) -- found with an atomic ticket, no waiting --
 // merges all partials with log-sum-exp weights (Metodologia 2: LSE-stabilised
 // merge) and writes the output.
+#include <mutex>
+
 #include "jl_common.cuh"
 #include "jl_ptx.cuh"
 
@@ -432,6 +434,119 @@ cudaError_t launch_decode(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t
     dl.tickets = reinterpret_cast<unsigned int*>(reinterpret_cast<unsigned char*>(p.workspace) + part);
     dl.dev_error = p.dev_error;
     cudaError_t e;
+    if (dt == JETLONG_FP32)
+        e = p.d == 64 ? launch_hpb<float, 64>(p, dl, s) : launch_hpb<float, 128>(p, dl, s);
+    else
+        e = p.d == 64 ? launch_hpb<__nv_bfloat16, 64>(p, dl, s)
+                      : launch_hpb<__nv_bfloat16, 128>(p, dl, s);
+    if (e == cudaSuccess) *nlaunch += 1;
+    return e;
+}
+
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  Some callers cannot allocate device memory at all:
+// code running under a caching allocator that must not grow, inside a host
+// callback, or in a runtime that hands this library only the tensors of the
+// step.  For them, jetlong_decode_noalloc runs the same split-K decode with its
+// scratch (the split partials and merge tickets) in the fixed array below
+// instead of a caller-provided workspace.  Every GPU that loads this library
+// holds the array until the process exits.  All calls on a device share it and
+// it keeps the last call's contents: the tickets are cleared at every call and
+// the partials are always written before they are read, so stale contents are
+// harmless, but two calls that overlap on the GPU (concurrent streams) race on
+// it and must be serialised by the caller.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[JETLONG_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the array, looked up once per device on the first call with
+// that device current.  Host code must not use the array's name as a pointer:
+// on the host it only names a stand-in for the symbol.
+void* noalloc_scratch_address(cudaError_t* err)
+{
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        *err = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
+// Split count that launch_typed<T, D, HPB> will pick for this problem (same
+// occupancy query and arithmetic).
+template <typename T, int D, int HPB>
+int planned_splits(const DecodeProblem& p, int hgroups, cudaError_t* err)
+{
+    auto kern = decode_split_kernel<T, D, HPB>;
+    constexpr int smem = decode_smem_bytes<T, D, HPB>();
+    *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (*err != cudaSuccess) return 0;
+    int dev = 0, nsm = 148, occ = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem);
+    if (occ < 1) occ = 1;
+    const int units = p.B * p.Hkv * hgroups;
+    int ns = (nsm * occ) / units;
+    ns = max(1, min(ns, max_splits(p.Lcap)));
+    ns = min(ns, max(1, (p.L + 63) / 64));
+    int chunk = (p.L + ns - 1) / ns;
+    chunk = (chunk + KROWS - 1) / KROWS * KROWS;
+    return (p.L + chunk - 1) / chunk;
+}
+
+template <typename T, int D>
+int planned_splits_hpb(const DecodeProblem& p, int hpb, int hgroups, cudaError_t* err)
+{
+    switch (hpb) {
+        case 4: return planned_splits<T, D, 4>(p, hgroups, err);
+        case 2: return planned_splits<T, D, 2>(p, hgroups, err);
+        default: return planned_splits<T, D, 1>(p, hgroups, err);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s,
+                                  int* nlaunch, size_t* need_bytes)
+{
+    *need_bytes = 0;
+    cudaError_t e;
+    unsigned char* scratch = static_cast<unsigned char*>(noalloc_scratch_address(&e));
+    if (!scratch) return e;
+    DecodeLaunch dl{};
+    const int group = p.Hq / p.Hkv;
+    dl.hpb = pick_hpb(group);
+    dl.hgroups = group / dl.hpb;
+    int ns;
+    if (dt == JETLONG_FP32)
+        ns = p.d == 64 ? planned_splits_hpb<float, 64>(p, dl.hpb, dl.hgroups, &e)
+                       : planned_splits_hpb<float, 128>(p, dl.hpb, dl.hgroups, &e);
+    else
+        ns = p.d == 64 ? planned_splits_hpb<__nv_bfloat16, 64>(p, dl.hpb, dl.hgroups, &e)
+                       : planned_splits_hpb<__nv_bfloat16, 128>(p, dl.hpb, dl.hgroups, &e);
+    if (ns < 1) return e;
+    size_t part = (size_t)p.B * p.Hq * ns * (p.d + 2) * sizeof(float);
+    part = (part + 255) / 256 * 256;
+    const size_t need = part + (size_t)p.B * p.Hkv * dl.hgroups * sizeof(unsigned int);
+    *need_bytes = need;
+    if (need > (size_t)JETLONG_DECODE_NOALLOC_SCRATCH_BYTES) return cudaErrorInvalidValue;
+    make_div_magic((uint32_t)p.G, &dl.div_m, &dl.div_s1, &dl.div_s2);
+    dl.partials = reinterpret_cast<float*>(scratch);
+    dl.tickets = reinterpret_cast<unsigned int*>(scratch + part);
+    dl.dev_error = p.dev_error;
     if (dt == JETLONG_FP32)
         e = p.d == 64 ? launch_hpb<float, 64>(p, dl, s) : launch_hpb<float, 128>(p, dl, s);
     else

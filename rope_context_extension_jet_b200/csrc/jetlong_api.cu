@@ -204,6 +204,45 @@ int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* 
     return ok();
 }
 
+int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* out,
+                           int B, int Hq, int Hkv, int L, int Lcap, int d, int w0,
+                           int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
+                           void* stream)
+{
+    if (!q || !kcache || !vcache || !out) return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out))
+        return fail(JETLONG_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if (L < 1 || Lcap < L)
+        return fail(JETLONG_ERR_INVALID_ARG, "need 1 <= L <= Lcap (L=%d Lcap=%d)", L, Lcap);
+    int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
+    if (st != JETLONG_OK) return st;
+    if ((int64_t)B * Hkv > 65535 * 64)
+        return fail(JETLONG_ERR_UNSUPPORTED, "B * Hkv too large");
+    cudaError_t e;
+    int* derr = dev_error_word(&e);
+    if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+
+    jl::DecodeProblem p{};
+    p.q = q; p.kc = kcache; p.vc = vcache; p.out = out;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.Lcap = Lcap; p.d = d;
+    p.w0 = w0 > L ? L : w0;
+    p.G = (int)jetlong_group_size(L, w_pretrained);
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    jl::make_rope_turns(&p.turns, d, rope_theta);
+    p.dev_error = derr;
+    int n = 0;
+    size_t need = 0;
+    e = jl::launch_decode_noalloc(p, dtype, (cudaStream_t)stream, &n, &need);
+    g_launches += n;
+    if (e == cudaErrorInvalidValue && need > (size_t)JETLONG_DECODE_NOALLOC_SCRATCH_BYTES)
+        return fail(JETLONG_ERR_INVALID_ARG,
+                    "decode needs %zu bytes of scratch; the fixed no-alloc array holds %u "
+                    "(use jetlong_decode with a workspace)",
+                    need, (unsigned)JETLONG_DECODE_NOALLOC_SCRATCH_BYTES);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 int jetlong_device_status(void* stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -106,6 +106,10 @@ cudaError_t launch_prefill_simt(const PrefillProblem& p, jetlong_dtype dt, cudaS
                                 int* nlaunch);
 cudaError_t launch_prefill_tc(const PrefillProblem& p, cudaStream_t s, int* nlaunch);
 cudaError_t launch_decode(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s, int* nlaunch);
+// Same decode with its scratch in the library's fixed device array; *need_bytes
+// receives the scratch this problem needs (cudaErrorInvalidValue if too large).
+cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s,
+                                  int* nlaunch, size_t* need_bytes);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d);
 cudaError_t launch_position_map(int32_t* out, int L, int G, cudaStream_t s, int* nlaunch);
 
