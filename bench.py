@@ -205,6 +205,32 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """One kernel on a reduced workload of the same shape family, for ncu."""
+    import torch
+    import rope_context_extension_jet_b200 as jl
+    jl.load_library()
+    torch.cuda.set_device(0)
+    if args.profile == "prefill":
+        w = I.C4.with_(L=args.L)
+        q, k, v = (to_dev(a, "cuda") for a in I.prefill_inputs(w))
+        out = torch.empty_like(q)
+        for _ in range(args.warmup + args.steps):
+            jl.prefill(q, k, v, out, w0=w.w0, w_pretrained=w.w_pretrained,
+                       rope_theta=w.rope_theta, scale=w.scale)
+    else:
+        w = I.D.with_(L0=args.L - 1, Lcap=args.L + 64, steps=1)
+        qs, kc, vc = I.decode_inputs(w)
+        qd, kcd, vcd = to_dev(np.ascontiguousarray(qs[0]), "cuda"), to_dev(kc, "cuda"), to_dev(vc, "cuda")
+        ws = torch.empty(jl.decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lcap, w.d), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(args.warmup + args.steps):
+            jl.decode(qd, kcd, vcd, w.length_at(0), w0=w.w0, w_pretrained=w.w_pretrained,
+                      rope_theta=w.rope_theta, scale=w.scale, workspace=ws)
+    jl.device_status()
+    print(json.dumps({"profile": args.profile, "L": args.L, "launches": jl.launch_count()}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -213,6 +239,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+                    help="run only one kernel on a reduced workload (for ncu captures)")
+    ap.add_argument("--L", type=int, default=32768, help="sequence / cache length for --profile")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -222,6 +251,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile:
+        run_profile(args)
         return
 
     import torch

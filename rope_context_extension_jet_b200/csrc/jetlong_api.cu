@@ -150,7 +150,9 @@ int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int 
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.dev_error = derr;
     int n = 0;
-    e = jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
+    // bf16: tensor-core kernel; fp32: CUDA-core fp32 kernel (TF32 would miss fp32 accuracy)
+    e = dtype == JETLONG_BF16 ? jl::launch_prefill_tc(p, (cudaStream_t)stream, &n)
+                              : jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
     return ok();
