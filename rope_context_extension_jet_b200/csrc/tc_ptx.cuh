@@ -95,6 +95,32 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
+// A from tensor memory: D[tmem] (+)= A[tmem] * B[smem]^T (kind::f16).  The A
+// tile (M = 128 rows = lanes, K = 16) occupies 8 consecutive 32-bit columns,
+// two 16-bit elements per column (even k in the low half).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Warpgroup register reallocation (all four warps of a warpgroup execute it).
+template <int N> __device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N> __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// Fast base-2 exponential (ex2.approx.ftz: ~2 ulp, flushes denormals; ex2(-inf) = 0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar)
 {
