@@ -17,6 +17,8 @@
 // the last CTA of a (b, kv head) -- found with an atomic ticket, no waiting --
 // merges all partials with log-sum-exp weights (Metodologia 2: LSE-stabilised
 // merge) and writes the output.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "jl_common.cuh"
@@ -95,6 +97,64 @@ __host__ __device__ constexpr int decode_smem_bytes()
                                                           : merge_bytes<D, HPB>())
            + 2 * HPB * D * 4        // rotated queries: [2][HPB][D]
            + 2 * DecodeCfg<T, D>::STAGES * 8 + 16;  // barriers + flag
+}
+
+// Merge the partial softmax states of the GROUPS lane groups (or warps) of this
+// CTA -- smem `mo` [HPB][GROUPS][D + 2] holding (o[D], max, sum) in base-2
+// units -- into the CTA's split partial in the workspace; the last CTA of this
+// (b, kv head, head group) to finish (atomic ticket, no waiting) then merges
+// all splits with log-sum-exp weights and writes the output rows.
+template <typename T, int D, int HPB, int GROUPS, int NTHR>
+__device__ void merge_splits(const float* mo, int* flag, const DecodeProblem& p, const DecodeLaunch& dl,
+                             int s, int b, int h0)
+{
+    const int tid = threadIdx.x;
+    float* part_out = dl.partials;
+    for (int e = tid; e < HPB * (D + 2); e += NTHR) {
+        const int hh = e / (D + 2), col = e % (D + 2);
+        float M = -INFINITY;
+        for (int grp = 0; grp < GROUPS; ++grp) M = fmaxf(M, mo[((size_t)hh * GROUPS + grp) * (D + 2) + D]);
+        float acc = 0.f;
+        if (M != -INFINITY) {
+            for (int grp = 0; grp < GROUPS; ++grp) {
+                const float* row = mo + ((size_t)hh * GROUPS + grp) * (D + 2);
+                if (row[D] == -INFINITY) continue;
+                const float w = exp2f(row[D] - M);
+                acc += w * (col == D ? 0.f : (col == D + 1 ? row[D + 1] : row[col]));
+            }
+        }
+        if (col == D) acc = M;
+        const size_t idx = (((size_t)b * p.Hq + h0 + hh) * dl.n_splits + s) * (D + 2) + col;
+        part_out[idx] = acc;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        unsigned int* tk = dl.tickets + (size_t)b * p.Hkv * dl.hgroups + blockIdx.y;
+        const unsigned int prev = atomicAdd(tk, 1u);
+        *flag = (prev == (unsigned int)dl.n_splits - 1) ? 1 : 0;
+        if (*flag) *tk = 0u;  // ready for the next call
+    }
+    __syncthreads();
+    if (*flag == 0) return;
+    __threadfence();
+    T* out = reinterpret_cast<T*>(p.out);
+    for (int e = tid; e < HPB * D; e += NTHR) {
+        const int hh = e / D, col = e % D;
+        const float* base = part_out + ((size_t)b * p.Hq + h0 + hh) * dl.n_splits * (D + 2);
+        float M = -INFINITY;
+        for (int sp = 0; sp < dl.n_splits; ++sp) M = fmaxf(M, __ldcg(base + (size_t)sp * (D + 2) + D));
+        float num = 0.f, den = 0.f;
+        for (int sp = 0; sp < dl.n_splits; ++sp) {
+            const float* row = base + (size_t)sp * (D + 2);
+            const float ms = __ldcg(row + D);
+            if (ms == -INFINITY) continue;
+            const float w = exp2f(ms - M);
+            num += w * __ldcg(row + col);
+            den += w * __ldcg(row + D + 1);
+        }
+        store_elem(out + ((size_t)b * p.Hq + h0 + hh) * D + col, num / den);
+    }
 }
 
 template <typename T, int D, int HPB>
@@ -305,52 +365,332 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
         }
     }
     __syncthreads();
-    float* part_out = dl.partials;
-    for (int e = tid; e < HPB * (D + 2); e += NT) {
-        const int hh = e / (D + 2), col = e % (D + 2);
-        float M = -INFINITY;
-        for (int grp = 0; grp < GROUPS; ++grp) M = fmaxf(M, mo[((size_t)hh * GROUPS + grp) * (D + 2) + D]);
-        float acc = 0.f;
-        if (M != -INFINITY) {
-            for (int grp = 0; grp < GROUPS; ++grp) {
-                const float* row = mo + ((size_t)hh * GROUPS + grp) * (D + 2);
-                if (row[D] == -INFINITY) continue;
-                const float w = exp2f(row[D] - M);
-                acc += w * (col == D ? 0.f : (col == D + 1 ? row[D + 1] : row[col]));
+    merge_splits<T, D, HPB, GROUPS, NT>(mo, flag, p, dl, s, b, h0);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 decode on warp-level tensor-core MMAs (m16n8k16).
+//
+// The group's query heads are the N = 8 columns of the MMA, 16 keys its M
+// rows: S^T (16 keys x 8 heads) = K_rot (16 x d) * Q_rot^T (d x 8), then
+// O^T (d x 8) += V^T (d x 16) * P^T (16 x 8).  K and V stream into shared
+// memory with 2-D TMA (128-byte swizzle, 64 keys per stage); each warp owns 16
+// keys of a stage: ldmatrix brings K fragments to registers, where the pairs
+// (m, m + d/2) sit in the same thread (k-steps kb and kb + d/32) and are
+// rotated to j or floor(j/G) before the MMA (fp16 operands; Q^T is fp16 too).
+// P goes through a 256-byte per-warp buffer to become the B fragment of P V.
+// Online softmax per head in base 2 with lazy rescaling (threshold 2^8).
+
+constexpr int TC_KROWS = 64, TC_NCW = 4, TC_NT = (TC_NCW + 1) * 32, TC_STAGES = 3;
+constexpr float kDecRescale = 8.0f;
+
+template <int D, int HPB>
+struct DecTcCfg {
+    static constexpr int ATOMS = D / 64;
+    static constexpr int TILE = TC_KROWS * D * 2;  // one K or V stage tile
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int RING = TC_STAGES * STAGE;
+    static constexpr int MERGE = HPB * TC_NCW * (D + 2) * 4;
+    static constexpr int BIG = RING > MERGE ? RING : MERGE;
+    static constexpr int PBUF = BIG;                       // [TC_NCW][16 keys][8 heads] bf16
+    static constexpr int SQ = PBUF + TC_NCW * 256;         // [2][HPB][D] fp32 rotated queries
+    static constexpr int TURNS = SQ + 2 * HPB * D * 4;     // [d/2] uint2 phase constants
+    static constexpr int BARS = TURNS + (D / 2) * 8;
+    static constexpr int END = BARS + 2 * TC_STAGES * 8 + 16;
+    static constexpr int TOTAL = END + 1024;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void tma_load_3d_dec(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// shared-memory address of 16-byte chunk `ch` of key row `key` in a stage tile
+// stored by TMA as [d/64 atoms][64 keys][128 B], chunk index XOR key % 8
+__device__ __forceinline__ uint32_t dec_sw(uint32_t tile, int key, int ch)
+{
+    return tile + (uint32_t)((ch >> 3) * (TC_KROWS * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4));
+}
+
+// S^T for the 16 keys of this warp's block: rotated K fragments times Q^T.
+template <int D>
+__device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int kw, int lane, uint32_t pa, uint32_t pb,
+                                             const uint2* sturns, const uint32_t (&qb)[D / 16][2])
+{
+    const int g = lane >> 2, t = lane & 3;
+    c[0] = c[1] = c[2] = c[3] = 0.f;
+    // ldmatrix.x4 rows: lanes 0-7 keys 0-7 / chunk lo, 8-15 keys 8-15 / lo, 16-23 keys 0-7 / hi, 24-31 keys 8-15 / hi
+    const int lkey = kw + (lane & 7) + ((lane >> 3) & 1) * 8, lhalf = lane >> 4;
+#pragma unroll
+    for (int kb = 0; kb < D / 32; ++kb) {
+        uint32_t lo[4], hi[4];
+        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + lhalf), lo);
+        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + D / 16 + lhalf), hi);
+        const int m0 = 16 * kb + 2 * t;
+        // lo[0]: key g, dims m0,m0+1; lo[1]: key g+8; lo[2]: key g, dims m0+8,m0+9; lo[3]: key g+8
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t pos = (r & 1) ? pb : pa;
+            const int m = m0 + ((r >> 1) ? 8 : 0);
+            const uint2 w0 = sturns[m], w1 = sturns[m + 1];
+            float c0, s0, c1, s1;
+            rope_cs_fast(pos, w0.x, w0.y, c0, s0);
+            rope_cs_fast(pos, w1.x, w1.y, c1, s1);
+            const float x0 = bf16_lo(lo[r]), x1 = bf16_hi(lo[r]);
+            const float y0 = bf16_lo(hi[r]), y1 = bf16_hi(hi[r]);
+            lo[r] = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+            hi[r] = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
+        }
+        mma_f16(c, lo, qb[kb][0], qb[kb][1]);
+        mma_f16(c, hi, qb[kb + D / 32][0], qb[kb + D / 32][1]);
+    }
+}
+
+template <int D, int HPB>
+__global__ void __launch_bounds__(TC_NT, 2)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     DecodeProblem p, DecodeLaunch dl)
+{
+    using C = DecTcCfg<D, HPB>;
+    constexpr int H = D / 2;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned char* ring = smem;
+    float* sq = reinterpret_cast<float*>(smem + C::SQ);           // [2][HPB][D]
+    uint2* sturns = reinterpret_cast<uint2*>(smem + C::TURNS);    // (hi, lo) per frequency
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BARS);
+    uint64_t* empty = full + TC_STAGES;
+    int* flag = reinterpret_cast<int*>(empty + TC_STAGES);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int s = blockIdx.x;
+    const int kvh = blockIdx.y / dl.hgroups, hg = blockIdx.y % dl.hgroups;
+    const int b = blockIdx.z;
+    const int group = p.Hq / p.Hkv;
+    const int h0 = kvh * group + hg * HPB;
+    const int L = p.L, i = L - 1;
+    const int j_begin = s * dl.chunk;
+    const int j_end = min(L, j_begin + dl.chunk);
+    const int nchunks = max(0, (j_end - j_begin + TC_KROWS - 1) / TC_KROWS);
+    const int j_exact = i - p.w0 + 1;  // keys j >= j_exact are local
+
+    if (tid == 0) {
+        for (int st = 0; st < TC_STAGES; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], TC_NCW);
+        }
+        fence_mbar_init();
+    }
+    for (int m = tid; m < H; m += TC_NT) sturns[m] = make_uint2(p.turns.hi[m], p.turns.lo[m]);
+    {
+        const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0) * D;
+        const uint32_t pe = (uint32_t)i, pr = div_g((uint32_t)i, dl);
+        for (int e = tid; e < HPB * H; e += TC_NT) {
+            const int hh = e / H, m = e % H;
+            const float a = load_elem(q + (size_t)hh * D + m), c2 = load_elem(q + (size_t)hh * D + m + H);
+            float c, sn;
+            rope_cs_accurate(pe, p.turns.hi[m], p.turns.lo[m], c, sn);
+            sq[(0 * HPB + hh) * D + m] = (a * c - c2 * sn) * p.scale_log2;
+            sq[(0 * HPB + hh) * D + m + H] = (a * sn + c2 * c) * p.scale_log2;
+            rope_cs_accurate(pr, p.turns.hi[m], p.turns.lo[m], c, sn);
+            sq[(1 * HPB + hh) * D + m] = (a * c - c2 * sn) * p.scale_log2;
+            sq[(1 * HPB + hh) * D + m + H] = (a * sn + c2 * c) * p.scale_log2;
+        }
+    }
+    __syncthreads();
+
+    const int zkv = b * p.Hkv + kvh;
+    float* mo = reinterpret_cast<float*>(ring);  // reused after the ring drains: [HPB][TC_NCW][D + 2]
+    if (warp == TC_NCW) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % TC_STAGES;
+                if (c >= TC_STAGES && !mbar_wait(&empty[st], ((c / TC_STAGES) - 1) & 1)) {
+                    record_error(dl.dev_error, 0x111);
+                    break;
+                }
+                const int j0 = j_begin + c * TC_KROWS;
+                unsigned char* dst = ring + st * C::STAGE;
+                mbar_arrive_expect_tx(&full[st], C::STAGE);
+#pragma unroll
+                for (int a = 0; a < C::ATOMS; ++a) {
+                    tma_load_3d_dec(dst + a * TC_KROWS * 128, &tmK, a * 64, j0, zkv, &full[st]);
+                    tma_load_3d_dec(dst + C::TILE + a * TC_KROWS * 128, &tmV, a * 64, j0, zkv, &full[st]);
+                }
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - TC_STAGES); c < issued; ++c)
+                if (!mbar_wait(&full[c % TC_STAGES], (c / TC_STAGES) & 1)) record_error(dl.dev_error, 0x112);
+        }
+        __syncthreads();
+    } else {
+        // ---------------------------------------------------------- consumers
+        const int g = lane >> 2, t = lane & 3;
+        // Q^T fragments (fp16): b0 = (Q[g][16kb+2t], Q[g][16kb+2t+1]), b1 = dims + 8; heads >= HPB are 0
+        uint32_t qb_ex[D / 16][2], qb_rm[D / 16][2];
+#pragma unroll
+        for (int kb = 0; kb < D / 16; ++kb) {
+            const int m = 16 * kb + 2 * t;
+            if (g < HPB) {
+                const float* qe = sq + (0 * HPB + g) * D;
+                const float* qr = sq + (1 * HPB + g) * D;
+                qb_ex[kb][0] = pack_f16x2(qe[m], qe[m + 1]);
+                qb_ex[kb][1] = pack_f16x2(qe[m + 8], qe[m + 9]);
+                qb_rm[kb][0] = pack_f16x2(qr[m], qr[m + 1]);
+                qb_rm[kb][1] = pack_f16x2(qr[m + 8], qr[m + 9]);
+            } else {
+                qb_ex[kb][0] = qb_ex[kb][1] = qb_rm[kb][0] = qb_rm[kb][1] = 0u;
             }
         }
-        if (col == D) acc = M;
-        const size_t idx = (((size_t)b * p.Hq + h0 + hh) * dl.n_splits + s) * (D + 2) + col;
-        part_out[idx] = acc;
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        unsigned int* tk = dl.tickets + (size_t)b * p.Hkv * dl.hgroups + blockIdx.y;
-        const unsigned int prev = atomicAdd(tk, 1u);
-        *flag = (prev == (unsigned int)dl.n_splits - 1) ? 1 : 0;
-        if (*flag) *tk = 0u;  // ready for the next call
-    }
-    __syncthreads();
-    if (*flag == 0) return;
-    __threadfence();
-    T* out = reinterpret_cast<T*>(p.out);
-    for (int e = tid; e < HPB * D; e += NT) {
-        const int hh = e / D, col = e % D;
-        const float* base = part_out + ((size_t)b * p.Hq + h0 + hh) * dl.n_splits * (D + 2);
-        float M = -INFINITY;
-        for (int sp = 0; sp < dl.n_splits; ++sp) M = fmaxf(M, __ldcg(base + (size_t)sp * (D + 2) + D));
-        float num = 0.f, den = 0.f;
-        for (int sp = 0; sp < dl.n_splits; ++sp) {
-            const float* row = base + (size_t)sp * (D + 2);
-            const float ms = __ldcg(row + D);
-            if (ms == -INFINITY) continue;
-            const float w = exp2f(ms - M);
-            num += w * __ldcg(row + col);
-            den += w * __ldcg(row + D + 1);
+        float o[D / 16][4];
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+        float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};  // heads 2t, 2t + 1
+        const uint32_t pbuf = smem_u32(smem + C::PBUF + warp * 256);
+        const int kw = warp * 16;  // this warp's keys within a stage
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % TC_STAGES;
+            if (!mbar_wait(&full[st], (c / TC_STAGES) & 1)) {
+                record_error(dl.dev_error, 0x113);
+                break;
+            }
+            const uint32_t ktile = smem_u32(ring + st * C::STAGE), vtile = ktile + C::TILE;
+            const int jb = j_begin + c * TC_KROWS + kw;  // first key of this warp's block
+            const int ja = jb + g, jc = jb + g + 8;     // the keys of rows g and g + 8
+            float sc[4];
+            if (jb >= j_exact) {
+                block_logits<D>(sc, ktile, kw, lane, (uint32_t)ja, (uint32_t)jc, sturns, qb_ex);
+            } else if (jb + 15 < j_exact) {
+                block_logits<D>(sc, ktile, kw, lane, div_g((uint32_t)ja, dl), div_g((uint32_t)jc, dl), sturns, qb_rm);
+            } else {
+                float se[4];
+                block_logits<D>(sc, ktile, kw, lane, div_g((uint32_t)ja, dl), div_g((uint32_t)jc, dl), sturns, qb_rm);
+                block_logits<D>(se, ktile, kw, lane, (uint32_t)ja, (uint32_t)jc, sturns, qb_ex);
+                if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
+                if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
+            }
+            if (ja >= j_end) sc[0] = sc[1] = -INFINITY;
+            if (jc >= j_end) sc[2] = sc[3] = -INFINITY;
+            // online softmax for heads 2t (sc[0], sc[2]) and 2t + 1 (sc[1], sc[3]) over the 16 keys
+            float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+                bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+            }
+            const float bm[2] = {bm0, bm1};
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float mn = fmaxf(mh[u], bm[u]);
+                if (mn > mh[u] + kDecRescale) {
+                    const float alpha = exp2f(mh[u] - mn);
+                    lh[u] *= alpha;
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        o[mt][u] *= alpha;
+                        o[mt][2 + u] *= alpha;
+                    }
+                    mh[u] = mn;
+                }
+            }
+            const float ms0 = mh[0] == -INFINITY ? 0.f : mh[0], ms1 = mh[1] == -INFINITY ? 0.f : mh[1];
+            const float p0 = exp2f(sc[0] - ms0), p1 = exp2f(sc[1] - ms1);
+            const float p2 = exp2f(sc[2] - ms0), p3 = exp2f(sc[3] - ms1);
+            lh[0] += p0 + p2;
+            lh[1] += p1 + p3;
+            // P^T fragment through the warp's buffer [16 keys][8 heads] bf16
+            __syncwarp();
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(pbuf + g * 16 + t * 4), "r"(pack_bf16x2(p0, p1)) : "memory");
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(pbuf + (g + 8) * 16 + t * 4), "r"(pack_bf16x2(p2, p3)) : "memory");
+            __syncwarp();
+            uint32_t pb0, pb1;
+            ldsm_x2_t(pbuf + (lane & 15) * 16, pb0, pb1);
+            // O^T += V^T P^T over the d/16 row tiles of 16 dims
+            const int vkey = kw + (lane & 7) + (lane >> 4) * 8, vhalf = (lane >> 3) & 1;
+#pragma unroll
+            // keys past the valid range (cache rows >= L may hold anything) contribute
+            // exactly zero: their V entries are cleared, not only their P
+            const bool tail = jb + 15 >= j_end;
+            const uint32_t m_lo = (jb + 2 * t < j_end ? 0x0000ffffu : 0u) | (jb + 2 * t + 1 < j_end ? 0xffff0000u : 0u);
+            const uint32_t m_hi = (jb + 2 * t + 8 < j_end ? 0x0000ffffu : 0u) | (jb + 2 * t + 9 < j_end ? 0xffff0000u : 0u);
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                uint32_t va[4];
+                ldsm_x4_t(dec_sw(vtile, vkey, 2 * mt + vhalf), va);
+                if (tail) {
+                    va[0] &= m_lo; va[1] &= m_lo; va[2] &= m_hi; va[3] &= m_hi;
+                }
+                mma_bf16(o[mt], va, pb0, pb1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
         }
-        store_elem(out + ((size_t)b * p.Hq + h0 + hh) * D + col, num / den);
+        // per-warp partial states -> smem [HPB][TC_NCW][D + 2]
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float lt = lh[u];
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, off);
+            lh[u] = lt;
+        }
+        __syncthreads();  // every warp finished with the ring
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int hh = 2 * t + u;
+            if (hh < HPB) {
+                float* row = mo + ((size_t)hh * TC_NCW + warp) * (D + 2);
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    row[16 * mt + g] = o[mt][u];
+                    row[16 * mt + g + 8] = o[mt][2 + u];
+                }
+                if (g == 0) {
+                    row[D] = mh[u];
+                    row[D + 1] = lh[u];
+                }
+            }
+        }
     }
+    __syncthreads();
+    merge_splits<__nv_bfloat16, D, HPB, TC_NCW, TC_NT>(mo, flag, p, dl, s, b, h0);
 }
 
 int pick_hpb(int group)
@@ -360,44 +700,134 @@ int pick_hpb(int group)
     return 1;
 }
 
+// heads per CTA for the tensor-core kernel: the MMA's N = 8 columns
+int pick_hpb_tc(int group)
+{
+    if (group % 8 == 0) return 8;
+    return pick_hpb(group);
+}
+
 int max_splits(int Lcap) { return min(kMaxSplits, max(1, (Lcap + 63) / 64)); }
 
-template <typename T, int D, int HPB>
-cudaError_t launch_typed(const DecodeProblem& p, DecodeLaunch dl, cudaStream_t st)
+// Split count and chunk length (a multiple of `gran` keys) for `units` CTAs'
+// worth of (b, kv head, head group) work: enough splits to fill every SM at the
+// kernel's occupancy, never more than the workspace holds.
+template <class Kern>
+cudaError_t plan_splits(const DecodeProblem& p, int units, Kern kern, int nthreads, int smem, int gran,
+                        int* ns_out, int* chunk_out)
 {
-    auto kern = decode_split_kernel<T, D, HPB>;
-    constexpr int smem = decode_smem_bytes<T, D, HPB>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148, occ = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads, smem);
     if (occ < 1) occ = 1;
-    const int units = p.B * p.Hkv * dl.hgroups;
     int ns = (nsm * occ) / units;
     ns = max(1, min(ns, max_splits(p.Lcap)));
     ns = min(ns, max(1, (p.L + 63) / 64));
     int chunk = (p.L + ns - 1) / ns;
-    chunk = (chunk + KROWS - 1) / KROWS * KROWS;
-    ns = (p.L + chunk - 1) / chunk;
-    dl.n_splits = ns;
-    dl.chunk = chunk;
-    // tickets live after the partials; zero them for this call
+    chunk = (chunk + gran - 1) / gran * gran;
+    *ns_out = (p.L + chunk - 1) / chunk;
+    *chunk_out = chunk;
+    return cudaSuccess;
+}
+
+template <typename T, int D, int HPB>
+cudaError_t plan_scalar(const DecodeProblem& p, DecodeLaunch& dl)
+{
+    return plan_splits(p, p.B * p.Hkv * dl.hgroups, decode_split_kernel<T, D, HPB>, NT,
+                       decode_smem_bytes<T, D, HPB>(), KROWS, &dl.n_splits, &dl.chunk);
+}
+
+template <int D, int HPB>
+cudaError_t plan_tc(const DecodeProblem& p, DecodeLaunch& dl)
+{
+    return plan_splits(p, p.B * p.Hkv * dl.hgroups, decode_tc_kernel<D, HPB>, TC_NT,
+                       DecTcCfg<D, HPB>::TOTAL, TC_KROWS, &dl.n_splits, &dl.chunk);
+}
+
+template <typename T, int D, int HPB>
+cudaError_t launch_scalar(const DecodeProblem& p, DecodeLaunch dl, cudaStream_t st)
+{
+    cudaError_t e = plan_scalar<T, D, HPB>(p, dl);
+    if (e != cudaSuccess) return e;
+    const int units = p.B * p.Hkv * dl.hgroups;
     e = cudaMemsetAsync(dl.tickets, 0, sizeof(unsigned int) * (size_t)units, st);
     if (e != cudaSuccess) return e;
-    dim3 grid(ns, p.Hkv * dl.hgroups, p.B);
-    kern<<<grid, NT, smem, st>>>(p, dl);
+    dim3 grid(dl.n_splits, p.Hkv * dl.hgroups, p.B);
+    decode_split_kernel<T, D, HPB><<<grid, NT, decode_smem_bytes<T, D, HPB>(), st>>>(p, dl);
     return cudaGetLastError();
 }
 
-template <typename T, int D>
-cudaError_t launch_hpb(const DecodeProblem& p, DecodeLaunch dl, cudaStream_t st)
+typedef CUresult (*EncodeTiledFnDec)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// [B*Hkv planes][Lcap rows][d] bf16, box 64 columns x 64 keys x 1 plane, 128-byte swizzle
+cudaError_t make_cache_map(CUtensorMap* m, const void* base, int d, int Lcap, int nplanes)
 {
+    static std::once_flag once;
+    static EncodeTiledFnDec fn = nullptr;
+    static cudaError_t st = cudaSuccess;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        st = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+        if (st == cudaSuccess && q != cudaDriverEntryPointSuccess) st = cudaErrorSymbolNotFound;
+        fn = reinterpret_cast<EncodeTiledFnDec>(f);
+    });
+    if (!fn) return st == cudaSuccess ? cudaErrorSymbolNotFound : st;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)Lcap, (cuuint64_t)nplanes};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)Lcap * d * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)TC_KROWS, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, int HPB>
+cudaError_t launch_tc(const DecodeProblem& p, DecodeLaunch dl, cudaStream_t st)
+{
+    CUtensorMap tk, tv;
+    cudaError_t e;
+    if ((e = make_cache_map(&tk, p.kc, D, p.Lcap, p.B * p.Hkv)) != cudaSuccess) return e;
+    if ((e = make_cache_map(&tv, p.vc, D, p.Lcap, p.B * p.Hkv)) != cudaSuccess) return e;
+    if ((e = plan_tc<D, HPB>(p, dl)) != cudaSuccess) return e;
+    const int units = p.B * p.Hkv * dl.hgroups;
+    e = cudaMemsetAsync(dl.tickets, 0, sizeof(unsigned int) * (size_t)units, st);
+    if (e != cudaSuccess) return e;
+    dim3 grid(dl.n_splits, p.Hkv * dl.hgroups, p.B);
+    decode_tc_kernel<D, HPB><<<grid, TC_NT, DecTcCfg<D, HPB>::TOTAL, st>>>(tk, tv, p, dl);
+    return cudaGetLastError();
+}
+
+// Head grouping and the split plan/launch for this problem's element type.
+void set_groups(const DecodeProblem& p, jetlong_dtype dt, DecodeLaunch& dl)
+{
+    const int group = p.Hq / p.Hkv;
+    dl.hpb = dt == JETLONG_BF16 ? pick_hpb_tc(group) : pick_hpb(group);
+    dl.hgroups = group / dl.hpb;
+}
+
+template <int D>
+cudaError_t dispatch(const DecodeProblem& p, jetlong_dtype dt, DecodeLaunch& dl, cudaStream_t st, bool plan_only)
+{
+    if (dt == JETLONG_FP32) {
+        switch (dl.hpb) {
+            case 4: return plan_only ? plan_scalar<float, D, 4>(p, dl) : launch_scalar<float, D, 4>(p, dl, st);
+            case 2: return plan_only ? plan_scalar<float, D, 2>(p, dl) : launch_scalar<float, D, 2>(p, dl, st);
+            default: return plan_only ? plan_scalar<float, D, 1>(p, dl) : launch_scalar<float, D, 1>(p, dl, st);
+        }
+    }
     switch (dl.hpb) {
-        case 4: return launch_typed<T, D, 4>(p, dl, st);
-        case 2: return launch_typed<T, D, 2>(p, dl, st);
-        default: return launch_typed<T, D, 1>(p, dl, st);
+        case 8: return plan_only ? plan_tc<D, 8>(p, dl) : launch_tc<D, 8>(p, dl, st);
+        case 4: return plan_only ? plan_tc<D, 4>(p, dl) : launch_tc<D, 4>(p, dl, st);
+        case 2: return plan_only ? plan_tc<D, 2>(p, dl) : launch_tc<D, 2>(p, dl, st);
+        default: return plan_only ? plan_tc<D, 1>(p, dl) : launch_tc<D, 1>(p, dl, st);
     }
 }
 
@@ -415,6 +845,7 @@ void make_div_magic(uint32_t G, uint32_t* m, uint32_t* s1, uint32_t* s2)
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d)
 {
+    // tickets are sized for the smaller of the two head groupings (more groups)
     const int hg = (Hq / Hkv) / pick_hpb(Hq / Hkv);
     size_t part = (size_t)B * Hq * max_splits(Lcap) * (d + 2) * sizeof(float);
     part = (part + 255) / 256 * 256;
@@ -424,25 +855,17 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d)
 cudaError_t launch_decode(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s, int* nlaunch)
 {
     DecodeLaunch dl{};
-    const int group = p.Hq / p.Hkv;
-    dl.hpb = pick_hpb(group);
-    dl.hgroups = group / dl.hpb;
+    set_groups(p, dt, dl);
     make_div_magic((uint32_t)p.G, &dl.div_m, &dl.div_s1, &dl.div_s2);
     size_t part = (size_t)p.B * p.Hq * max_splits(p.Lcap) * (p.d + 2) * sizeof(float);
     part = (part + 255) / 256 * 256;
     dl.partials = reinterpret_cast<float*>(p.workspace);
     dl.tickets = reinterpret_cast<unsigned int*>(reinterpret_cast<unsigned char*>(p.workspace) + part);
     dl.dev_error = p.dev_error;
-    cudaError_t e;
-    if (dt == JETLONG_FP32)
-        e = p.d == 64 ? launch_hpb<float, 64>(p, dl, s) : launch_hpb<float, 128>(p, dl, s);
-    else
-        e = p.d == 64 ? launch_hpb<__nv_bfloat16, 64>(p, dl, s)
-                      : launch_hpb<__nv_bfloat16, 128>(p, dl, s);
+    cudaError_t e = p.d == 64 ? dispatch<64>(p, dt, dl, s, false) : dispatch<128>(p, dt, dl, s, false);
     if (e == cudaSuccess) *nlaunch += 1;
     return e;
 }
-
 
 // ---------------------------------------------------------------------------
 // Allocation-free decode.  Some callers cannot allocate device memory at all:
@@ -484,39 +907,6 @@ void* noalloc_scratch_address(cudaError_t* err)
     return addr[dev];
 }
 
-// Split count that launch_typed<T, D, HPB> will pick for this problem (same
-// occupancy query and arithmetic).
-template <typename T, int D, int HPB>
-int planned_splits(const DecodeProblem& p, int hgroups, cudaError_t* err)
-{
-    auto kern = decode_split_kernel<T, D, HPB>;
-    constexpr int smem = decode_smem_bytes<T, D, HPB>();
-    *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (*err != cudaSuccess) return 0;
-    int dev = 0, nsm = 148, occ = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem);
-    if (occ < 1) occ = 1;
-    const int units = p.B * p.Hkv * hgroups;
-    int ns = (nsm * occ) / units;
-    ns = max(1, min(ns, max_splits(p.Lcap)));
-    ns = min(ns, max(1, (p.L + 63) / 64));
-    int chunk = (p.L + ns - 1) / ns;
-    chunk = (chunk + KROWS - 1) / KROWS * KROWS;
-    return (p.L + chunk - 1) / chunk;
-}
-
-template <typename T, int D>
-int planned_splits_hpb(const DecodeProblem& p, int hpb, int hgroups, cudaError_t* err)
-{
-    switch (hpb) {
-        case 4: return planned_splits<T, D, 4>(p, hgroups, err);
-        case 2: return planned_splits<T, D, 2>(p, hgroups, err);
-        default: return planned_splits<T, D, 1>(p, hgroups, err);
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t s,
@@ -527,18 +917,11 @@ cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cuda
     unsigned char* scratch = static_cast<unsigned char*>(noalloc_scratch_address(&e));
     if (!scratch) return e;
     DecodeLaunch dl{};
-    const int group = p.Hq / p.Hkv;
-    dl.hpb = pick_hpb(group);
-    dl.hgroups = group / dl.hpb;
-    int ns;
-    if (dt == JETLONG_FP32)
-        ns = p.d == 64 ? planned_splits_hpb<float, 64>(p, dl.hpb, dl.hgroups, &e)
-                       : planned_splits_hpb<float, 128>(p, dl.hpb, dl.hgroups, &e);
-    else
-        ns = p.d == 64 ? planned_splits_hpb<__nv_bfloat16, 64>(p, dl.hpb, dl.hgroups, &e)
-                       : planned_splits_hpb<__nv_bfloat16, 128>(p, dl.hpb, dl.hgroups, &e);
-    if (ns < 1) return e;
-    size_t part = (size_t)p.B * p.Hq * ns * (p.d + 2) * sizeof(float);
+    set_groups(p, dt, dl);
+    // the split count the launch below will use (same planner, same kernel)
+    e = p.d == 64 ? dispatch<64>(p, dt, dl, s, true) : dispatch<128>(p, dt, dl, s, true);
+    if (e != cudaSuccess) return e;
+    size_t part = (size_t)p.B * p.Hq * dl.n_splits * (p.d + 2) * sizeof(float);
     part = (part + 255) / 256 * 256;
     const size_t need = part + (size_t)p.B * p.Hkv * dl.hgroups * sizeof(unsigned int);
     *need_bytes = need;
@@ -547,11 +930,7 @@ cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cuda
     dl.partials = reinterpret_cast<float*>(scratch);
     dl.tickets = reinterpret_cast<unsigned int*>(scratch + part);
     dl.dev_error = p.dev_error;
-    if (dt == JETLONG_FP32)
-        e = p.d == 64 ? launch_hpb<float, 64>(p, dl, s) : launch_hpb<float, 128>(p, dl, s);
-    else
-        e = p.d == 64 ? launch_hpb<__nv_bfloat16, 64>(p, dl, s)
-                      : launch_hpb<__nv_bfloat16, 128>(p, dl, s);
+    e = p.d == 64 ? dispatch<64>(p, dt, dl, s, false) : dispatch<128>(p, dt, dl, s, false);
     if (e == cudaSuccess) *nlaunch += 1;
     return e;
 }

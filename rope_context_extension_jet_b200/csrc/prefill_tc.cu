@@ -52,6 +52,7 @@ namespace {
 
 constexpr int BM = 128, BN = 128, NSK = 2, NSV = 2, NTHREADS = 512;
 constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
+constexpr long long kTcWaitCycles = 1000000000ll;  // ~0.5 s: every wait here is on work of this CTA
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
@@ -109,7 +110,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > kTcWaitCycles) {
             record_error(dev_error, code);
             *abort_flag = 1;
             return false;
@@ -216,6 +217,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int i_hi = min(qb * BM + BM - 1, L - 1);
     const int nkb = i_hi / BN + 1;
 
+    // after a bounded wait expired anywhere in the grid (error word set), later
+    // CTAs skip their work so a failed launch ends quickly; the host reads and
+    // clears the word with jetlong_device_status
+    if (*reinterpret_cast<volatile int*>(p.dev_error) != 0) return;
     if (tid == 0) {
         mbar_init(&bars[B_QFULL], 1);
         mbar_init(&bars[B_QREADY0], 4);
