@@ -69,6 +69,22 @@ def decode_bytes(w, L):
     return kv, kv + qo
 
 
+def prefill_traffic():
+    """DRAM bytes per 128K prefill launch from the committed ncu capture, or None
+    when the kernel source changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)["prefill_tc_kernel"]
+        src = os.path.join(ROOT, "rope_context_extension_jet_b200", "csrc", "prefill_tc.cu")
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return rec["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -396,12 +412,19 @@ def main():
                        "gbs_kv": round(dec_gbs, 1), "bytes_per_pass_kv": kv_bytes,
                        "bytes_per_pass_all": all_bytes, "tokens_per_s": round(dec_tok_s, 1),
                        "frac_of_hbm": round(dec_gbs / world / peaks["hbm_gbs"], 4),
+                       "roofline": {"bound": "hbm", "achieved": round(dec_gbs / world, 1),
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(dec_gbs / world / peaks["hbm_gbs"], 4),
+                                    "kernel": "decode_tc_kernel<128, 4>",
+                                    "peak_source": f"{peaks['source']} HBM copy"},
                        "G": [jl.group_size(wd.length_at(0), wd.w_pretrained),
                              jl.group_size(wd.length_at(wd.steps - 1), wd.w_pretrained)]},
             "roofline": {"bound": "tensor", "achieved": round(pre_tflops / world, 2),
                          "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": round(frac_s, 4), "traffic": None,
-                         "peak_source": f"{peaks['source']} bf16 sustained"},
+                         "frac": round(frac_s, 4), "traffic": prefill_traffic(),
+                         "kernel": "prefill_tc_kernel<128, 2>",
+                         "peak_source": f"{peaks['source']} bf16 sustained (the prefill "
+                                        "runs ~170 ms at a time inside a ~220 ms step)"},
             "e2e": {"value": round(world * computed / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
