@@ -195,6 +195,14 @@ def oracle_prefill_sample(w, budget_s=20.0, nthreads=0):
                       f"fp64, useful FLOPs 4*d*(i+1) per row"}
 
 
+def bench_config(wp, wd, world):
+    """The `config` object of the JSON line (identical for both arms)."""
+    return {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d, "L": wp.L,
+            "w_pretrained": wp.w_pretrained, "G": max(1, -(-wp.L // wp.w_pretrained)),
+            "w0": wp.w0, "rope_theta": wp.rope_theta, "decode_workload": wd.name,
+            "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -212,13 +220,29 @@ def run_reference(args, rank, world):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs * 1000.0 / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L": w.L,
-                   "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.rope_theta},
+        "config": bench_config(w, I.D, world),
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": steps[0]["cores"],
                          "kind": "oracle", "sample": steps[0]["sample"]},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def max_across_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the multi-GPU timing rule: a
+    replica job takes as long as its slowest rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput of `world` replicas: all ranks' work / slowest rank's time."""
+    return world * work_per_rank / max_seconds
 
 
 def run_profile(args):
@@ -289,11 +313,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_across_ranks(x, world, dev)
 
     peaks = load_peaks()
     wp, wd = I.C4, I.D
@@ -358,12 +378,12 @@ def main():
     dec_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev_d])))
 
     useful, computed, tiles, band = prefill_flops(wp)
-    pre_tflops = world * computed / (pre_ms * 1e-3) / 1e12
-    pre_useful_tflops = world * useful / (pre_ms * 1e-3) / 1e12
+    pre_tflops = whole_job_rate(computed, world, pre_ms * 1e-3) / 1e12
+    pre_useful_tflops = whole_job_rate(useful, world, pre_ms * 1e-3) / 1e12
     kv_bytes = sum(decode_bytes(wd, wd.length_at(t))[0] for t in range(wd.steps))
     all_bytes = sum(decode_bytes(wd, wd.length_at(t))[1] for t in range(wd.steps))
-    dec_gbs = world * kv_bytes / (dec_ms * 1e-3) / 1e9
-    dec_tok_s = world * wd.B * wd.steps / (dec_ms * 1e-3)
+    dec_gbs = whole_job_rate(kv_bytes, world, dec_ms * 1e-3) / 1e9
+    dec_tok_s = whole_job_rate(wd.B * wd.steps, world, dec_ms * 1e-3)
 
     # ---------------- end to end through the public API with host buffers
     qh, kh, vh = to_pinned(q), to_pinned(k), to_pinned(v)
@@ -396,11 +416,7 @@ def main():
             "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) q/k/v, bf16)",
-            "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d,
-                       "L": wp.L, "w_pretrained": wp.w_pretrained, "G": jl.group_size(wp.L, wp.w_pretrained),
-                       "w0": wp.w0, "rope_theta": wp.rope_theta,
-                       "decode_workload": wd.name, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (no flush)"},
+            "config": bench_config(wp, wd, world),
             "prefill": {"ms": round(pre_ms, 3), "tflops_computed": round(pre_tflops, 2),
                         "tflops_useful": round(pre_useful_tflops, 2),
                         "flops_computed": computed, "flops_useful": useful,

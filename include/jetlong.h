@@ -129,6 +129,15 @@ int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache
  * JETLONG_ERR_CUDA. */
 int jetlong_device_status(void* stream);
 
+/* Self test of the failure-detection path (the pages have no counterpart):
+ * launches one small kernel that waits on a barrier nothing arrives at, using
+ * the same bounded-wait helper as the attention kernels with a ~1 ms limit.
+ * The wait expires, the kernel sets the device error word and returns, so the
+ * next jetlong_device_status(stream) reports JETLONG_ERR_TIMEOUT (and clears
+ * the word).  No fault, no hang; the context stays usable.  Returns
+ * JETLONG_OK or JETLONG_ERR_CUDA (launch failure). */
+int jetlong_selftest_wait_timeout(void* stream);
+
 /* Message for the last failing call on this host thread ("" if none). */
 const char* jetlong_last_error(void);
 

@@ -22,7 +22,7 @@ import threading
 __all__ = [
     "BF16", "FP32", "JetLongError", "load_library", "group_size", "position_map", "prefill",
     "decode_workspace_size", "decode", "decode_noalloc", "device_status", "last_error",
-    "launch_count", "DECODE_NOALLOC_SCRATCH_BYTES",
+    "launch_count", "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,8 @@ def load_library(path: str | None = None):
         lib.jetlong_decode_noalloc.restype = i32
         lib.jetlong_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                                i32, dbl, flt, i32, vp]
+        lib.jetlong_selftest_wait_timeout.restype = i32
+        lib.jetlong_selftest_wait_timeout.argtypes = [vp]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -209,6 +211,12 @@ def decode_noalloc(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained
                                       int(w_pretrained), float(rope_theta), float(scale),
                                       _dtype_code(q), _stream(stream)), lib)
     return out
+
+
+def selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait self test; the next device_status() raises TIMEOUT."""
+    lib = load_library()
+    _check(lib.jetlong_selftest_wait_timeout(_stream(stream)), lib)
 
 
 def device_status(stream=None):

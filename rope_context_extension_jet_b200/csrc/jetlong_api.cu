@@ -245,6 +245,18 @@ int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache
     return ok();
 }
 
+int jetlong_selftest_wait_timeout(void* stream)
+{
+    cudaError_t e;
+    int* derr = dev_error_word(&e);
+    if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+    int n = 0;
+    e = jl::launch_wait_selftest(derr, 2000000ll, (cudaStream_t)stream, &n);  // ~1 ms
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 int jetlong_device_status(void* stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -119,5 +119,6 @@ cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cuda
                                   int* nlaunch, size_t* need_bytes);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d);
 cudaError_t launch_position_map(int32_t* out, int L, int G, cudaStream_t s, int* nlaunch);
+cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStream_t s, int* nlaunch);
 
 }  // namespace jl

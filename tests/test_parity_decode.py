@@ -98,3 +98,22 @@ def test_workspace_contents_do_not_matter():
     ws.fill_(0x5A)
     b = run_decode(w, qs, kc, vc, [0], ws=ws)[0]
     np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_cache_rows_past_length_are_ignored(dtype):
+    """Rows >= L of the caches may hold anything (here NaN): the output must not see them."""
+    import torch
+    w = small_decode("dec-nan-tail", dtype=dtype, L0=1000, Lcap=1100, steps=1, index=46)
+    qs, kc, vc = I.decode_inputs(w)
+    L = w.length_at(0)
+    kd, vd = to_device(kc), to_device(vc)
+    kd[:, :, L:] = float("nan")
+    vd[:, :, L:] = float("nan")
+    qd = to_device(np.ascontiguousarray(qs[0]))
+    out = jl.decode(qd, kd, vd, L, w0=w.w0, w_pretrained=w.w_pretrained, rope_theta=w.rope_theta,
+                    scale=w.scale)
+    jl.device_status()
+    ref = oracle.decode(np.ascontiguousarray(qs[0]), kc, vc, L, w0=w.w0,
+                        w_pretrained=w.w_pretrained, rope_theta=w.rope_theta, scale=w.scale)
+    check_gate(to_host_f64(out), ref, dtype, "decode with NaN rows past L")
