@@ -69,17 +69,29 @@ def decode_bytes(w, L):
     return kv, kv + qo
 
 
+PREFILL_KERNEL = "prefill_pair_kernel"
+# sources the timed prefill kernel is compiled from (its DRAM counters are
+# reported only while they hash to the value recorded with the capture)
+PREFILL_SOURCES = ("prefill_pair.cu", "prefill_tc_common.cuh", "tc_ptx.cuh", "jl_ptx.cuh", "jl_common.cuh")
+
+
+def prefill_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for name in PREFILL_SOURCES:
+        with open(os.path.join(ROOT, "rope_context_extension_jet_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def prefill_traffic():
     """DRAM bytes per 128K prefill launch from the committed ncu capture, or None
-    when the kernel source changed since the counters were taken."""
-    import hashlib
+    when the kernel sources changed since the counters were taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)["prefill_tc_kernel"]
-        src = os.path.join(ROOT, "rope_context_extension_jet_b200", "csrc", "prefill_tc.cu")
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+            rec = json.load(f)[PREFILL_KERNEL]
+        if prefill_source_hash() != rec["source_sha256"]:
+            return None
         return rec["dram_bytes_per_launch"]
     except (OSError, KeyError, ValueError):
         return None
@@ -438,7 +450,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": round(pre_tflops / world, 2),
                          "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": round(frac_s, 4), "traffic": prefill_traffic(),
-                         "kernel": "prefill_tc_kernel<128, 2>",
+                         "kernel": PREFILL_KERNEL,
                          "peak_source": f"{peaks['source']} bf16 sustained (the prefill "
                                         "runs ~170 ms at a time inside a ~220 ms step)"},
             "e2e": {"value": round(world * computed / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",

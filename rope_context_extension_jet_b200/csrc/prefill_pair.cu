@@ -1,0 +1,333 @@
+// prefill_pair.cu -- bf16 prefill of dynamic bifocal RoPE attention (d = 128)
+// on CTA pairs: every tensor-core MMA spans the two SMs of a cluster pair
+// (tcgen05 cta_group::2, M = 256).
+//
+// "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
+// (gist.science/it/paper/2607.07740), Metodologia 1-2: local pairs
+// (i - j < w0) are rotated at (i, j), remote pairs at (floor(i/G), floor(j/G)),
+// rotations applied on the fly to the raw inputs, one softmax for both.
+//
+// Work unit of a pair: one block of 128 query rows of the four query heads
+// that share a kv head.  CTA r (r = 0, 1) holds heads 2r and 2r + 1 of the four:
+// their Q tiles, S and O in its own TMEM (lanes = query rows).  A K tile (128
+// keys) is split by keys: CTA r loads and rotates keys [64r, 64r + 64); a V tile
+// is split by columns: CTA r loads V[:, 64r, 64r + 64).  One MMA
+//   S_h = Q_h K^T : A = Q_h of both CTAs (M = 256), B = both K halves (N = 128)
+//   O_h += P_h V  : A = P_h in both TMEMs, B = both V halves (N = d)
+// so each SM stages and rotates half of every K/V tile, and reads half of the
+// B operand from its shared memory, while the MMA rate per SM is unchanged.
+// The phases, masks and softmax are those of the one-CTA kernel
+// (prefill_tc.cu): phase R (remote and band tiles, aliased positions), then
+// phase E (band and local tiles, exact positions), Q re-rotated in between.
+//
+// Roles (512 threads per CTA; registers rebalanced with setmaxnreg):
+//   warp 0      TMA producer (both CTAs): own Q tiles, own K and V halves
+//   warp 1      MMA issuer (CTA 0 only, one thread), cta_group::2
+//   warp 2      TMEM allocation / release (cta_group::2, both CTAs)
+//   warp 3      CTA 1: tells CTA 0 when its V half landed
+//   warps 4-7   rotation of own Q tiles and own K halves
+//   warps 8-15  softmax, heads 2r (8-11) and 2r + 1 (12-15)
+// Synchronisation: CTA 0's MMA thread waits on barriers in CTA 0 that both CTAs
+// arrive on (Q and K rotated, P written, V halves landed); its commits arrive
+// on the barriers at the same offset in both CTAs (S ready, P.V done, buffers
+// free).  Every wait is bounded; on expiry a CTA records an error code, stops,
+// and both CTAs meet at the closing cluster barrier before TMEM is released.
+#include "prefill_tc_common.cuh"
+
+namespace jl {
+namespace tc {
+namespace {
+
+constexpr int D = 128;
+constexpr int NS = 4;           // ring depth of the K and V halves
+constexpr int KROWS = BN / 2;   // keys of a K tile held by one CTA
+constexpr int NTHREADS = 512;
+
+enum {
+    P_QFULL = 0, P_QREADY0, P_QREADY1, P_QFREE,
+    P_KFULL, P_KREADY = P_KFULL + NS, P_KEMPTY = P_KREADY + NS,
+    P_VFULL = P_KEMPTY + NS, P_VPEER = P_VFULL + NS, P_VEMPTY = P_VPEER + NS,
+    P_SFULL = P_VEMPTY + NS, P_PFULL = P_SFULL + 2, P_PVDONE = P_PFULL + 2,
+    P_DRAIN = P_PVDONE + 2, P_NBARS
+};
+
+struct PairSmem {
+    static constexpr int QTILE = BM * D * 2;      // 128 rows x 128 d: 2 atoms of 16 KB
+    static constexpr int KATOM = KROWS * 128;     // 64 rows x 64 columns
+    static constexpr int KTILE = KROWS * D * 2;   // 64 keys x 128 d: 2 atoms of 8 KB
+    static constexpr int VTILE = BN * 64 * 2;     // 128 keys x 64 columns: 1 atom
+    static constexpr int K0 = 2 * QTILE;
+    static constexpr int V0 = K0 + NS * KTILE;
+    static constexpr int BAR = V0 + NS * VTILE;
+    static constexpr int END = BAR + P_NBARS * 8 + 32;
+    static constexpr int TOTAL = END + 1024;      // slack to align the base to 1024
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const TcParams p)
+{
+    using S = PairSmem;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_NBARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* skip_word = reinterpret_cast<int*>(tmem_slot + 2);
+    TilePlan* plan = reinterpret_cast<TilePlan*>(tmem_slot + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int qb = p.nqb - 1 - (int)(blockIdx.x >> 1);  // heaviest query blocks first
+    const int hq4 = blockIdx.y * 4;                      // first of the pair's four query heads
+    const int h0 = hq4 + 2 * (int)rank;                  // this CTA's two heads
+    const int b = blockIdx.z;
+    const int kvh = hq4 / (p.Hq / p.Hkv);
+    // barriers of CTA 0, as cluster addresses (both CTAs arrive on them)
+    const uint32_t lbar = mapa_shared(smem_u32(bars), 0);
+    auto lead = [&](int idx) { return lbar + 8u * (uint32_t)idx; };
+
+    if (tid == 0) {
+        mbar_init(&bars[P_QFULL], 1);
+        mbar_init(&bars[P_QREADY0], 8);
+        mbar_init(&bars[P_QREADY1], 8);
+        mbar_init(&bars[P_QFREE], 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&bars[P_KFULL + s], 1);
+            mbar_init(&bars[P_KREADY + s], 8);
+            mbar_init(&bars[P_KEMPTY + s], 1);
+            mbar_init(&bars[P_VFULL + s], 1);
+            mbar_init(&bars[P_VPEER + s], 1);
+            mbar_init(&bars[P_VEMPTY + s], 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bars[P_SFULL + h], 1);
+            mbar_init(&bars[P_PFULL + h], 8);
+            mbar_init(&bars[P_PVDONE + h], 1);
+        }
+        mbar_init(&bars[P_DRAIN], 1);
+        *abort_flag = 0;
+        *plan = plan_tiles(qb, p.L, p.w0);
+        // after a bounded wait expired anywhere in the grid (error word set),
+        // later pairs skip their work; CTA 0 decides for both
+        if (leader) *skip_word = *reinterpret_cast<volatile int*>(p.dev_error) != 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, CTA 0's decision visible
+    const bool skip = ld_shared_cluster_u32(mapa_shared(smem_u32(skip_word), 0)) != 0;
+    if (!skip && warp == 2) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+        tc_fence_before();
+    }
+    __syncthreads();
+    cluster_sync();  // no CTA reads the other's shared memory before this point is passed
+    if (skip) return;
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const TilePlan tp = *plan;
+    const int nR = tp.nR, NE = tp.count();
+
+    if (warp < 4) {
+        regs_dec<56>();
+        if (warp == 0 && lane == 0) {
+            // ---------------------------------------------------------- TMA producer
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const int zkv = b * p.Hkv + kvh;
+            mbar_arrive_expect_tx(&bars[P_QFULL], 2 * S::QTILE);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+                    tma_load_3d(smem + h * S::QTILE + a * ATOM, &tmQ, a * 64, qb * BM, b * p.Hq + h0 + h,
+                                &bars[P_QFULL]);
+            int k_issued = 0, v_issued = 0;
+            for (int e = 0; e < NE; ++e) {
+                const int kb = tp.kb(e);
+                const int s = e % NS, u = e / NS;
+                if (e >= NS && !wait_or_abort<true>(&bars[P_KEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, 0x401)) break;
+                mbar_arrive_expect_tx(&bars[P_KFULL + s], S::KTILE);
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+                    tma_load_3d(smem + S::K0 + s * S::KTILE + a * S::KATOM, &tmK, a * 64, kb * BN + (int)rank * KROWS,
+                                zkv, &bars[P_KFULL + s]);
+                k_issued = e + 1;
+                if (e >= NS && !wait_or_abort<true>(&bars[P_VEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, 0x402)) break;
+                mbar_arrive_expect_tx(&bars[P_VFULL + s], S::VTILE);
+                tma_load_3d(smem + S::V0 + s * S::VTILE, &tmV, (int)rank * 64, kb * BN, zkv, &bars[P_VFULL + s]);
+                v_issued = e + 1;
+            }
+            // drain: the copies this thread issued have landed before the CTA exits
+            mbar_wait(&bars[P_QFULL], 0);
+            for (int ee = max(0, k_issued - NS); ee < k_issued; ++ee) mbar_wait(&bars[P_KFULL + ee % NS], (ee / NS) & 1);
+            for (int ee = max(0, v_issued - NS); ee < v_issued; ++ee) mbar_wait(&bars[P_VFULL + ee % NS], (ee / NS) & 1);
+        } else if (warp == 1 && lane == 0 && leader) {
+            // ---------------------------------------------------------- MMA issuer
+            constexpr uint32_t IDESC_QK = idesc_f16(2 * BM, BN, 0);
+            constexpr uint32_t IDESC_PV = idesc_bf16(2 * BM, D, 1);
+            const uint32_t sbase = smem_u32(smem);
+            auto qk = [&](int h, int s) {
+                const uint32_t qaddr = sbase + h * S::QTILE, kaddr = sbase + S::K0 + s * S::KTILE;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k)
+                    umma_pair_ss(tmem + h * 128, sdesc_sw128(qaddr + (k >> 2) * ATOM + (k & 3) * 32, 16, 1024),
+                                 sdesc_sw128(kaddr + (k >> 2) * S::KATOM + (k & 3) * 32, 16, 1024), IDESC_QK,
+                                 k > 0 ? 1u : 0u);
+                umma_commit_pair_both(&bars[P_SFULL + h]);
+            };
+            auto pv = [&](int h, int s, bool first) {
+                const uint32_t vaddr = sbase + S::V0 + s * S::VTILE;
+#pragma unroll
+                for (int k = 0; k < BN / 16; ++k)
+                    umma_pair_ts(tmem + 256 + h * 128, tmem + h * 128 + k * 8,
+                                 sdesc_sw128(vaddr + k * 2048, S::VTILE, 1024), IDESC_PV, (!first || k > 0) ? 1u : 0u);
+                umma_commit_pair_both(&bars[P_PVDONE + h]);
+            };
+            // V half of tile pe landed in both CTAs and P_h of tile pe is in both TMEMs
+            auto pv_ready = [&](int h, int pe) {
+                const int s = pe % NS, u = pe / NS;
+                return wait_or_abort<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, 0x411 + h) &&
+                       (h == 1 || (wait_or_abort(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x413) &&
+                                   wait_or_abort<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, 0x414)));
+            };
+            // Issue order per tile e: P_0 V (tile e-1), Q_0 K^T (tile e), P_1 V
+            // (tile e-1), Q_1 K^T (tile e).  S_h(e) overwrites P_h(e-1) in TMEM;
+            // the P.V reading it was issued earlier by this thread and the
+            // tensor pipe runs one thread's MMAs in issue order.
+            bool ok = wait_or_abort<true>(&bars[P_QREADY0], 0, abort_flag, p.dev_error, 0x415);
+            tc_fence_after();
+            for (int e = 0; e < NE && ok; ++e) {
+                const int s = e % NS, u = e / NS, pe = e - 1, ps = (e + NS - 1) % NS;
+                if (e > 0) {
+                    if (!pv_ready(0, pe)) { ok = false; break; }
+                    tc_fence_after();
+                    pv(0, ps, pe == 0);
+                }
+                if (e == nR && nR > 0) {
+                    // Q of phase R is no longer read once every MMA so far completed
+                    umma_commit_pair_both(&bars[P_QFREE]);
+                    if (!wait_or_abort<true>(&bars[P_QREADY1], 0, abort_flag, p.dev_error, 0x416)) { ok = false; break; }
+                }
+                if (!wait_or_abort<true>(&bars[P_KREADY + s], u & 1, abort_flag, p.dev_error, 0x417)) { ok = false; break; }
+                tc_fence_after();
+                qk(0, s);
+                if (e > 0) {
+                    if (!pv_ready(1, pe)) { ok = false; break; }
+                    tc_fence_after();
+                    pv(1, ps, pe == 0);
+                    umma_commit_pair_both(&bars[P_VEMPTY + ps]);
+                }
+                qk(1, s);
+                umma_commit_pair_both(&bars[P_KEMPTY + s]);
+            }
+            if (ok && NE > 0) {
+                const int pe = NE - 1, ps = pe % NS;
+                if (pv_ready(0, pe)) {
+                    tc_fence_after();
+                    pv(0, ps, pe == 0);
+                    if (pv_ready(1, pe)) {
+                        tc_fence_after();
+                        pv(1, ps, pe == 0);
+                        umma_commit_pair_both(&bars[P_VEMPTY + ps]);
+                    }
+                }
+            }
+            // drain: every MMA issued by this thread completed before the pair
+            // meets at the closing cluster barrier
+            umma_commit_pair_local(&bars[P_DRAIN]);
+            mbar_wait(&bars[P_DRAIN], 0);
+        } else if (warp == 3 && lane == 0 && !leader) {
+            // ---------------------------------------------------------- V relay (CTA 1)
+            for (int e = 0; e < NE; ++e) {
+                const int s = e % NS, u = e / NS;
+                if (!wait_or_abort(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x421)) break;
+                mbar_arrive_cluster(lead(P_VPEER + s));
+            }
+        }
+    } else if (warp < 8) {
+        regs_dec<88>();
+        // -------------------------------------------------------------- rotation
+        const int t = tid - 128;
+        float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
+        rope_steps<D>(t, p, stc, sts);
+        const uint32_t i0 = (uint32_t)(qb * BM);
+        bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, 0x431);
+        if (ok) {
+            for (int h = 0; h < 2; ++h) {
+                if (nR > 0)
+                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
+                else
+                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead(P_QREADY0));
+        }
+        for (int e = 0; e < NE && ok; ++e) {
+            const int kb = tp.kb(e);
+            const int s = e % NS, u = e / NS;
+            if (e == nR && nR > 0) {
+                // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
+                if (!warp_wait<true>(&bars[P_QFREE], 0, abort_flag, p.dev_error, 0x432)) { ok = false; break; }
+                for (int h = 0; h < 2; ++h)
+                    rotate_tile<D, BM, false>(smem + h * S::QTILE, t, p,
+                                              [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(lead(P_QREADY1));
+            }
+            if (!warp_wait(&bars[P_KFULL + s], u & 1, abort_flag, p.dev_error, 0x433)) { ok = false; break; }
+            const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
+            unsigned char* kt = smem + S::K0 + s * S::KTILE;
+            if (e < nR)
+                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
+            else
+                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead(P_KREADY + s));
+        }
+    } else {
+        regs_inc<184>();
+        // -------------------------------------------------------------- softmax (head hh)
+        const int hh = (warp - 8) >> 2;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint32_t pfull = lead(P_PFULL + hh);
+        softmax_role<D, true>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128, lane_base + 256 + hh * 128,
+                              &bars[P_SFULL + hh], &bars[P_PVDONE + hh], [pfull] { mbar_arrive_cluster(pfull); },
+                              abort_flag);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the pair's MMAs, copies and remote arrivals are over in both CTAs
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
+{
+    CUtensorMap tq, tk, tv;
+    cudaError_t e;
+    if ((e = make_map(&tq, pp.q, D, pp.L, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, pp.k, D, pp.L, pp.B * pp.Hkv, KROWS)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, pp.v, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    const TcParams p = make_params(pp);
+    constexpr int smem = PairSmem::TOTAL;
+    if ((e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    dim3 grid(2 * p.nqb, pp.Hq / 4, pp.B);
+    prefill_pair_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace jl

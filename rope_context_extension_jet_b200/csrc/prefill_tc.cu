@@ -39,38 +39,20 @@
 // Every mbarrier wait is bounded; on expiry the CTA records an error code in
 // the library's device error word, stops, drains its own copies and MMAs with
 // bounded waits, frees TMEM and returns.
-#include <cuda.h>
-
-#include <mutex>
-
-#include "jl_common.cuh"
-#include "jl_ptx.cuh"
-#include "tc_ptx.cuh"
+#include "prefill_tc_common.cuh"
 
 namespace jl {
+namespace tc {
 namespace {
 
-constexpr int BM = 128, BN = 128, NSK = 2, NSV = 2, NTHREADS = 512;
-constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
-constexpr long long kTcWaitCycles = 1000000000ll;  // ~0.5 s: every wait here is on work of this CTA
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+constexpr int NSK = 2, NSV = 2, NTHREADS = 512;
 
-enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
 enum {
     B_QFULL = 0, B_QREADY0, B_QREADY1, B_QFREE,
     B_KFULL, B_KREADY = B_KFULL + NSK, B_KEMPTY = B_KREADY + NSK,
     B_VFULL = B_KEMPTY + NSK, B_VEMPTY = B_VFULL + NSV,
     B_SFULL = B_VEMPTY + NSV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
     B_DRAIN = B_PVDONE + 2, NBARS
-};
-
-struct TcParams {
-    int B, Hq, Hkv, L, w0, G, nqb;
-    uint32_t div_m, div_s1, div_s2;  // floor(x / G) by multiply-shift
-    float scale_log2;
-    RopeTurns turns;
-    __nv_bfloat16* out;
-    int* dev_error;
 };
 
 template <int D, int NH>
@@ -84,117 +66,6 @@ struct TcSmem {
     static constexpr int TOTAL = END + 1024;  // slack to align the base to 1024
 };
 
-__device__ __forceinline__ uint32_t div_g(uint32_t n, const TcParams& p)
-{
-    // Granlund & Montgomery, "Division by Invariant Integers using
-    // Multiplication" (1994), Fig. 4.1: exact for all 32-bit n.
-    const uint32_t t1 = __umulhi(p.div_m, n);
-    return (t1 + ((n - t1) >> p.div_s1)) >> p.div_s2;
-}
-
-__device__ __forceinline__ int tile_class(int qb, int kb, int L, int w0)
-{
-    const int i_lo = qb * BM, i_hi = min(qb * BM + BM - 1, L - 1);
-    const int dmax = i_hi - kb * BN;
-    const int dmin = max(0, i_lo - (kb * BN + BN - 1));
-    if (dmax < w0) return CLS_LOC;
-    if (dmin >= w0) return CLS_REM;
-    return CLS_BAND;
-}
-
-// Bounded wait that also gives up once another role of the CTA aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int* dev_error, int code)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kTcWaitCycles) {
-            record_error(dev_error, code);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-    return true;
-}
-
-// Warp-collective form: every lane polls, and the warp proceeds only if all did.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* dev_error, int code)
-{
-    const bool ok = wait_or_abort(bar, parity, abort_flag, dev_error, code);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Byte offset of 16-byte chunk `ch` (8 16-bit columns, ch < d/8) of row r in a
-// 128-row tile stored as [d/64 atoms][128 rows][128 B] with the 128-byte swizzle
-// (chunk index XOR row % 8): the layout TMA writes and UMMA K-major reads.
-__device__ __forceinline__ uint32_t sw128_off(int r, int ch)
-{
-    return (uint32_t)((ch >> 3) * ATOM + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ float f16_lo(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu))); }
-__device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
-
-// RoPE of a 128-row tile in place (pairs (m, m + d/2)), output fp16.  Thread t
-// of the 128 rotation threads owns 8 frequencies (chunk c) of RPT consecutive
-// rows.  pos(row) must step by 0 or 1 between consecutive rows (true for j,
-// floor(j/G) and i - floor(i/G)); the angles of the first row come from the
-// exact fixed-point phase, later rows advance by the per-frequency step
-// rotation R(theta_m) (any other step is recomputed exactly).
-template <int D, bool IN_BF16, class PosFn>
-__device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const TcParams& p, PosFn pos,
-                                            const float (&stc)[8], const float (&sts)[8])
-{
-    constexpr int H = D / 2, CH = H / 8, RPT = CH;  // 128 threads = CH chunks x (128 / RPT) row groups
-    const int c = t % CH, row0 = (t / CH) * RPT;
-    float cs[8], sn[8];
-    uint32_t prev = pos(row0);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) rope_cs_fast(prev, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
-#pragma unroll 2
-    for (int s = 0; s < RPT; ++s) {
-        const int r = row0 + s;
-        if (s > 0) {
-            const uint32_t cur = pos(r);
-            if (cur == prev + 1) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float c2 = cs[u] * stc[u] - sn[u] * sts[u];
-                    sn[u] = sn[u] * stc[u] + cs[u] * sts[u];
-                    cs[u] = c2;
-                }
-            } else if (cur != prev) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) rope_cs_fast(cur, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
-            }
-            prev = cur;
-        }
-        uint4* plo = reinterpret_cast<uint4*>(tile + sw128_off(r, c));
-        uint4* phi = reinterpret_cast<uint4*>(tile + sw128_off(r, c + CH));
-        const uint4 a = *plo, bq = *phi;
-        const uint32_t la[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t lb[4] = {bq.x, bq.y, bq.z, bq.w};
-        uint32_t oa[4], ob[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            float x0, x1, y0, y1;
-            if (IN_BF16) {
-                x0 = bf16_lo(la[w]); x1 = bf16_hi(la[w]); y0 = bf16_lo(lb[w]); y1 = bf16_hi(lb[w]);
-            } else {
-                x0 = f16_lo(la[w]); x1 = f16_hi(la[w]); y0 = f16_lo(lb[w]); y1 = f16_hi(lb[w]);
-            }
-            const int u0 = 2 * w, u1 = 2 * w + 1;
-            oa[w] = pack_f16x2(x0 * cs[u0] - y0 * sn[u0], x1 * cs[u1] - y1 * sn[u1]);
-            ob[w] = pack_f16x2(x0 * sn[u0] + y0 * cs[u0], x1 * sn[u1] + y1 * cs[u1]);
-        }
-        *plo = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        *phi = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-    }
-}
-
 template <int D, int NH>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -207,15 +78,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* plan = reinterpret_cast<int*>(tmem_slot + 2);  // nR, kE0
+    TilePlan* plan = reinterpret_cast<TilePlan*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qb = p.nqb - 1 - (int)blockIdx.x;  // heaviest query blocks first
     const int h0 = blockIdx.y * NH, b = blockIdx.z;
     const int kvh = h0 / (p.Hq / p.Hkv);
-    const int L = p.L;
-    const int i_hi = min(qb * BM + BM - 1, L - 1);
-    const int nkb = i_hi / BN + 1;
 
     // after a bounded wait expired anywhere in the grid (error word set), later
     // CTAs skip their work so a failed launch ends quickly; the host reads and
@@ -242,15 +110,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
-        // phase R = tiles [0, nR) (classes REM, BAND); phase E = [kE0, nkb) (BAND, LOC)
-        int nR = nkb, kE0 = nkb;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int cls = tile_class(qb, kb, L, p.w0);
-            if (cls != CLS_REM && kE0 == nkb) kE0 = kb;
-            if (cls == CLS_LOC) { nR = kb; break; }
-        }
-        plan[0] = nR;
-        plan[1] = kE0;
+        *plan = plan_tiles(qb, p.L, p.w0);
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -261,9 +121,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int nR = plan[0], kE0 = plan[1];
-    const int NE = nR + (nkb - kE0);
-    auto kb_of = [&](int e) { return e < nR ? e : kE0 + (e - nR); };
+    const TilePlan tp = *plan;
+    const int nR = tp.nR, NE = tp.count();
 
     if (warp < 4) {
         regs_dec<56>();
@@ -281,7 +140,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                 &bars[B_QFULL]);
             int k_issued = 0, v_issued = 0;
             for (int e = 0; e < NE; ++e) {
-                const int kb = kb_of(e);
+                const int kb = tp.kb(e);
                 const int sk = e % NSK, uk = e / NSK;
                 if (e >= NSK && !wait_or_abort(&bars[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, p.dev_error, 0x301)) break;
                 mbar_arrive_expect_tx(&bars[B_KFULL + sk], S::TILE);
@@ -375,32 +234,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         regs_dec<88>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
-        constexpr int CH = D / 16;
-        const int c = t % CH;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) rope_cs_fast(1u, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], stc[u], sts[u]);
+        rope_steps<D>(t, p, stc, sts);
         const uint32_t i0 = (uint32_t)(qb * BM);
         bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, 0x321);
         if (ok) {
             for (int h = 0; h < NH; ++h) {
                 if (nR > 0)
-                    rotate_tile<D, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
                 else
-                    rotate_tile<D, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_QREADY0]);
         }
         for (int e = 0; e < NE && ok; ++e) {
-            const int kb = kb_of(e);
+            const int kb = tp.kb(e);
             const int sk = e % NSK, uk = e / NSK;
             if (e == nR && nR > 0) {
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
                 if (!warp_wait(&bars[B_QFREE], 0, abort_flag, p.dev_error, 0x322)) { ok = false; break; }
                 for (int h = 0; h < NH; ++h)
-                    rotate_tile<D, false>(smem + h * S::TILE, t, p,
+                    rotate_tile<D, BM, false>(smem + h * S::TILE, t, p,
                                           [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts);
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -409,9 +265,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, 0x323)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN);
             if (e < nR)
-                rotate_tile<D, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
+                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
             else
-                rotate_tile<D, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts);
+                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_KREADY + sk]);
@@ -421,119 +277,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // -------------------------------------------------------------- softmax (head hh)
         const int hh = (warp - 8) >> 2;
         if (hh < NH) {
-            const int r = tid & 127;
-            const int i = qb * BM + r;
             const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-            const uint32_t s_col = lane_base + hh * 128, o_col = lane_base + 256 + hh * 128;
-            const float sl2 = p.scale_log2;
-            float m_used = -INFINITY, l = 0.f;
-            bool ok = true;
-            for (int e = 0; e < NE; ++e) {
-                const int kb = kb_of(e);
-                const bool phase_r = e < nR;
-                const int cls = tile_class(qb, kb, L, p.w0);
-                if (!warp_wait(&bars[B_SFULL + hh], e & 1, abort_flag, p.dev_error, 0x331)) { ok = false; break; }
-                tc_fence_after();
-                float x[BN];
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t tt[32];
-                    tmem_ld32(s_col + cc * 32, tt);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) x[cc * 32 + u] = __uint_as_float(tt[u]);
-                }
-                const int j0 = kb * BN;
-                const bool need_mask = (j0 + BN - 1 > qb * BM) || (j0 + BN > L) || cls == CLS_BAND;
-                if (need_mask) {
-                    const int dw = i - j0 - p.w0;  // pair (i, j0 + u) is local iff u > dw
-#pragma unroll
-                    for (int u = 0; u < BN; ++u) {
-                        const int j = j0 + u;
-                        bool masked = (j > i) || (j >= L);
-                        if (cls == CLS_BAND) masked = masked || (phase_r ? (u > dw) : (u <= dw));
-                        if (masked) x[u] = -INFINITY;
-                    }
-                }
-                float m4[4] = {x[0], x[1], x[2], x[3]};
-#pragma unroll
-                for (int u = 4; u < BN; u += 4) {
-                    m4[0] = fmaxf(m4[0], x[u]);
-                    m4[1] = fmaxf(m4[1], x[u + 1]);
-                    m4[2] = fmaxf(m4[2], x[u + 2]);
-                    m4[3] = fmaxf(m4[3], x[u + 3]);
-                }
-                const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-                const float m_new = fmaxf(m_used, mt);
-                const bool resc = m_new > m_used + kRescaleThreshold;
-                float alpha = 1.f;
-                if (resc) {
-                    alpha = ex2_approx(m_used - m_new);
-                    m_used = m_new;
-                    l *= alpha;
-                }
-                const float ms = m_used == -INFINITY ? 0.f : m_used;
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[BN / 2];
-#pragma unroll
-                for (int u = 0; u < BN; u += 2) {
-                    const float p0 = ex2_approx(fmaf(x[u], sl2, -ms));
-                    const float p1 = ex2_approx(fmaf(x[u + 1], sl2, -ms));
-                    l4[(u >> 1) & 3] += p0 + p1;
-                    pk[u >> 1] = pack_bf16x2(p0, p1);
-                }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-                if (e > 0) {
-                    // previous P.V of this head finished: O is stable and P's columns are free
-                    if (!warp_wait(&bars[B_PVDONE + hh], (e - 1) & 1, abort_flag, p.dev_error, 0x332)) { ok = false; break; }
-                    tc_fence_after();
-                    if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t tt[32];
-                            tmem_ld32(o_col + cc * 32, tt);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int u = 0; u < 32; ++u) tt[u] = __float_as_uint(__uint_as_float(tt[u]) * alpha);
-                            tmem_st32(o_col + cc * 32, tt);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int cc = 0; cc < BN / 64; ++cc) {
-                    uint32_t tt[32];
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) tt[u] = pk[cc * 32 + u];
-                    tmem_st32(s_col + cc * 32, tt);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_PFULL + hh]);
-            }
-            // epilogue: O / l -> bf16 -> out
-            if (ok && NE > 0 && warp_wait(&bars[B_PVDONE + hh], (NE - 1) & 1, abort_flag, p.dev_error, 0x333)) {
-                tc_fence_after();
-                const float inv = 1.f / l;
-                __nv_bfloat16* orow = p.out + (((size_t)b * p.Hq + h0 + hh) * (size_t)L + (size_t)i) * D;
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t tt[32];
-                    tmem_ld32(o_col + cc * 32, tt);
-                    tmem_wait_ld();
-                    if (i < L) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(tt[q * 8 + 0]) * inv, __uint_as_float(tt[q * 8 + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(tt[q * 8 + 2]) * inv, __uint_as_float(tt[q * 8 + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(tt[q * 8 + 4]) * inv, __uint_as_float(tt[q * 8 + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(tt[q * 8 + 6]) * inv, __uint_as_float(tt[q * 8 + 7]) * inv);
-                            *reinterpret_cast<uint4*>(orow + cc * 32 + q * 8) = v;
-                        }
-                    }
-                }
-            }
+            uint64_t* pfull = &bars[B_PFULL + hh];
+            softmax_role<D, false>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128,
+                                   lane_base + 256 + hh * 128, &bars[B_SFULL + hh], &bars[B_PVDONE + hh],
+                                   [pfull] { mbar_arrive(pfull); }, abort_flag);
         }
     }
     tc_fence_before();
@@ -545,6 +293,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // --------------------------------------------------------------------- host
+
+template <int D, int NH>
+cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
+{
+    CUtensorMap tq, tk, tv;
+    cudaError_t e;
+    if ((e = make_map(&tq, pp.q, D, pp.L, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, pp.k, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, pp.v, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    const TcParams p = make_params(pp);
+    auto kern = prefill_tc_kernel<D, NH>;
+    constexpr int smem = TcSmem<D, NH>::TOTAL;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+        return e;
+    dim3 grid(p.nqb, pp.Hq / NH, pp.B);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -567,22 +333,6 @@ EncodeTiledFn encode_fn(cudaError_t* err)
     return fn;
 }
 
-// [planes][L rows][d] bf16, box 64 columns x 128 rows x 1 plane, 128-byte swizzle.
-cudaError_t make_map(CUtensorMap* m, const void* base, int d, int L, int nplanes)
-{
-    cudaError_t err;
-    EncodeTiledFn fn = encode_fn(&err);
-    if (!fn) return err == cudaSuccess ? cudaErrorSymbolNotFound : err;
-    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)nplanes};
-    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)BM, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 void make_div_magic(uint32_t G, uint32_t* m, uint32_t* s1, uint32_t* s2)
 {
     uint32_t l = 0;
@@ -592,14 +342,25 @@ void make_div_magic(uint32_t G, uint32_t* m, uint32_t* s1, uint32_t* s2)
     *s2 = l > 1 ? l - 1 : 0;
 }
 
-template <int D, int NH>
-cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
+}  // namespace
+
+cudaError_t make_map(CUtensorMap* m, const void* base, int d, int L, int nplanes, int box_rows)
 {
-    CUtensorMap tq, tk, tv;
-    cudaError_t e;
-    if ((e = make_map(&tq, pp.q, D, pp.L, pp.B * pp.Hq)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, pp.k, D, pp.L, pp.B * pp.Hkv)) != cudaSuccess) return e;
-    if ((e = make_map(&tv, pp.v, D, pp.L, pp.B * pp.Hkv)) != cudaSuccess) return e;
+    cudaError_t err;
+    EncodeTiledFn fn = encode_fn(&err);
+    if (!fn) return err == cudaSuccess ? cudaErrorSymbolNotFound : err;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)nplanes};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+TcParams make_params(const PrefillProblem& pp)
+{
     TcParams p{};
     p.B = pp.B; p.Hq = pp.Hq; p.Hkv = pp.Hkv; p.L = pp.L; p.w0 = pp.w0; p.G = pp.G;
     p.nqb = (pp.L + BM - 1) / BM;
@@ -608,25 +369,24 @@ cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
     p.turns = pp.turns;
     p.out = reinterpret_cast<__nv_bfloat16*>(pp.out);
     p.dev_error = pp.dev_error;
-    auto kern = prefill_tc_kernel<D, NH>;
-    constexpr int smem = TcSmem<D, NH>::TOTAL;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-        return e;
-    dim3 grid(p.nqb, pp.Hq / NH, pp.B);
-    kern<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    return p;
 }
 
-}  // namespace
+}  // namespace tc
 
+// d = 128 with a multiple of four query heads per kv head: CTA pairs sharing
+// every MMA (prefill_pair.cu); otherwise one CTA per 128 query rows of one or
+// two heads of a kv head.
 cudaError_t launch_prefill_tc(const PrefillProblem& p, cudaStream_t s, int* nlaunch)
 {
-    const bool pair = ((p.Hq / p.Hkv) % 2) == 0;  // two query heads of one kv head per CTA
+    const int group = p.Hq / p.Hkv;
     cudaError_t e;
-    if (p.d == 64)
-        e = pair ? launch_d<64, 2>(p, s) : launch_d<64, 1>(p, s);
+    if (p.d == 128 && group % 4 == 0)
+        e = tc::launch_prefill_pair(p, s);
+    else if (p.d == 64)
+        e = group % 2 == 0 ? tc::launch_d<64, 2>(p, s) : tc::launch_d<64, 1>(p, s);
     else
-        e = pair ? launch_d<128, 2>(p, s) : launch_d<128, 1>(p, s);
+        e = group % 2 == 0 ? tc::launch_d<128, 2>(p, s) : tc::launch_d<128, 1>(p, s);
     if (e == cudaSuccess) *nlaunch += 1;
     return e;
 }

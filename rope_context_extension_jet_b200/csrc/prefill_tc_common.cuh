@@ -1,0 +1,348 @@
+// prefill_tc_common.cuh -- pieces shared by the two tensor-core prefill kernels
+// of dynamic bifocal RoPE attention (one CTA per work unit in prefill_tc.cu, a
+// CTA pair sharing every MMA in prefill_pair.cu): tile classification, the
+// floor(x / G) division, bounded barrier waits, the in-place RoPE of a swizzled
+// shared-memory tile, the softmax role and the host-side TMA descriptors.
+//
+// "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
+// (gist.science/it/paper/2607.07740), Metodologia 1-2: a pair (i, j) with
+// i - j < w0 is rotated at (i, j), every other pair at (floor(i/G), floor(j/G));
+// both branches feed one softmax.
+#pragma once
+
+#include <cuda.h>
+
+#include <mutex>
+
+#include "jl_common.cuh"
+#include "jl_ptx.cuh"
+#include "tc_ptx.cuh"
+
+namespace jl {
+namespace tc {
+
+constexpr int BM = 128, BN = 128;
+constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
+constexpr long long kTcWaitCycles = 1000000000ll;  // ~0.5 s: every wait here is on work of this CTA (pair)
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
+
+struct TcParams {
+    int B, Hq, Hkv, L, w0, G, nqb;
+    uint32_t div_m, div_s1, div_s2;  // floor(x / G) by multiply-shift
+    float scale_log2;
+    RopeTurns turns;
+    __nv_bfloat16* out;
+    int* dev_error;
+};
+
+__device__ __forceinline__ uint32_t div_g(uint32_t n, const TcParams& p)
+{
+    // Granlund & Montgomery, "Division by Invariant Integers using
+    // Multiplication" (1994), Fig. 4.1: exact for all 32-bit n.
+    const uint32_t t1 = __umulhi(p.div_m, n);
+    return (t1 + ((n - t1) >> p.div_s1)) >> p.div_s2;
+}
+
+// Class of the (query block qb, key block kb) tile: every pair local, every
+// pair remote, or both (the band i - j = w0 crosses the tile).
+__device__ __forceinline__ int tile_class(int qb, int kb, int L, int w0)
+{
+    const int i_lo = qb * BM, i_hi = min(qb * BM + BM - 1, L - 1);
+    const int dmax = i_hi - kb * BN;
+    const int dmin = max(0, i_lo - (kb * BN + BN - 1));
+    if (dmax < w0) return CLS_LOC;
+    if (dmin >= w0) return CLS_REM;
+    return CLS_BAND;
+}
+
+// Key tiles of query block qb in processing order: phase R = [0, nR) (remote
+// and band tiles, rotated at the aliased positions), then phase E = [kE0, nkb)
+// (band and local tiles, rotated at the exact positions).
+struct TilePlan {
+    int nR, kE0, nkb;
+    __device__ __forceinline__ int count() const { return nR + (nkb - kE0); }
+    __device__ __forceinline__ int kb(int e) const { return e < nR ? e : kE0 + (e - nR); }
+};
+
+__device__ __forceinline__ TilePlan plan_tiles(int qb, int L, int w0)
+{
+    TilePlan t;
+    t.nkb = min(qb * BM + BM - 1, L - 1) / BN + 1;
+    t.nR = t.nkb;
+    t.kE0 = t.nkb;
+    for (int kb = 0; kb < t.nkb; ++kb) {
+        const int cls = tile_class(qb, kb, L, w0);
+        if (cls != CLS_REM && t.kE0 == t.nkb) t.kE0 = kb;
+        if (cls == CLS_LOC) { t.nR = kb; break; }
+    }
+    return t;
+}
+
+template <bool CLUSTER>
+__device__ __forceinline__ bool bar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+}
+
+// Bounded wait that also gives up once another role of the CTA aborted.  The
+// CLUSTER form acquires at cluster scope (the phase was completed by arrivals
+// or MMA commits from the other CTA of a pair).
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int* dev_error, int code)
+{
+    if (bar_try_wait<CLUSTER>(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!bar_try_wait<CLUSTER>(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kTcWaitCycles) {
+            record_error(dev_error, code);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// Warp-collective form: every lane polls, and the warp proceeds only if all did.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* dev_error, int code)
+{
+    const bool ok = wait_or_abort<CLUSTER>(bar, parity, abort_flag, dev_error, code);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Byte offset of 16-byte chunk `ch` (8 16-bit columns, ch < d/8) of row r in a
+// ROWS-row tile stored as [d/64 atoms][ROWS rows][128 B] with the 128-byte
+// swizzle (chunk index XOR row % 8): the layout TMA writes and UMMA K-major reads.
+template <int ROWS>
+__device__ __forceinline__ uint32_t sw128_off(int r, int ch)
+{
+    return (uint32_t)((ch >> 3) * (ROWS * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
+
+// RoPE of a ROWS-row tile in place (pairs (m, m + d/2)), output fp16.  Thread t
+// of the 128 rotation threads owns 8 frequencies (chunk c) of RPT consecutive
+// rows.  pos(row) must step by 0 or 1 between consecutive rows (true for j,
+// floor(j/G) and i - floor(i/G)); the angles of the first row come from the
+// exact fixed-point phase, later rows advance by the per-frequency step
+// rotation R(theta_m) (any other step is recomputed exactly).
+template <int D, int ROWS, bool IN_BF16, class PosFn>
+__device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const TcParams& p, PosFn pos,
+                                            const float (&stc)[8], const float (&sts)[8])
+{
+    constexpr int H = D / 2, CH = H / 8, RPT = ROWS * CH / 128;  // 128 threads = CH chunks x (ROWS / RPT) row groups
+    static_assert(RPT >= 1 && ROWS * CH == 128 * RPT, "rotation thread mapping");
+    const int c = t % CH, row0 = (t / CH) * RPT;
+    float cs[8], sn[8];
+    uint32_t prev = pos(row0);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) rope_cs_fast(prev, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+#pragma unroll 2
+    for (int s = 0; s < RPT; ++s) {
+        const int r = row0 + s;
+        if (s > 0) {
+            const uint32_t cur = pos(r);
+            if (cur == prev + 1) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float c2 = cs[u] * stc[u] - sn[u] * sts[u];
+                    sn[u] = sn[u] * stc[u] + cs[u] * sts[u];
+                    cs[u] = c2;
+                }
+            } else if (cur != prev) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) rope_cs_fast(cur, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+            }
+            prev = cur;
+        }
+        uint4* plo = reinterpret_cast<uint4*>(tile + sw128_off<ROWS>(r, c));
+        uint4* phi = reinterpret_cast<uint4*>(tile + sw128_off<ROWS>(r, c + CH));
+        const uint4 a = *plo, bq = *phi;
+        const uint32_t la[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t lb[4] = {bq.x, bq.y, bq.z, bq.w};
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            float x0, x1, y0, y1;
+            if (IN_BF16) {
+                x0 = bf16_lo(la[w]); x1 = bf16_hi(la[w]); y0 = bf16_lo(lb[w]); y1 = bf16_hi(lb[w]);
+            } else {
+                x0 = f16_lo(la[w]); x1 = f16_hi(la[w]); y0 = f16_lo(lb[w]); y1 = f16_hi(lb[w]);
+            }
+            const int u0 = 2 * w, u1 = 2 * w + 1;
+            oa[w] = pack_f16x2(x0 * cs[u0] - y0 * sn[u0], x1 * cs[u1] - y1 * sn[u1]);
+            ob[w] = pack_f16x2(x0 * sn[u0] + y0 * cs[u0], x1 * sn[u1] + y1 * cs[u1]);
+        }
+        *plo = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *phi = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+}
+
+// Per-frequency one-position step rotation R(theta_m) of rotation thread t.
+template <int D>
+__device__ __forceinline__ void rope_steps(int t, const TcParams& p, float (&stc)[8], float (&sts)[8])
+{
+    const int c = t % (D / 16);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) rope_cs_fast(1u, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], stc[u], sts[u]);
+}
+
+// Softmax role of one query head: one thread per query row (= TMEM lane), 4
+// warps.  For each key tile e: wait for S = Q K^T in TMEM (`sfull`), apply the
+// causal / length / band masks, online softmax in base 2 with lazy O rescaling
+// (once the previous P.V finished, `pvdone`), write P (bf16) over the first 64
+// columns of S and signal the MMA issuer (`arrive_p`); finally O / l -> out.
+// s_col / o_col are this warp's TMEM addresses of S and O.
+template <int D, bool CLUSTER, class ArriveP>
+__device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& tp, int qb, int head, int b,
+                                             int r, uint32_t s_col, uint32_t o_col, uint64_t* sfull,
+                                             uint64_t* pvdone, ArriveP arrive_p, volatile int* abort_flag)
+{
+    const int lane = r & 31;
+    const int L = p.L;
+    const int i = qb * BM + r;
+    const int NE = tp.count();
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int e = 0; e < NE; ++e) {
+        const int kb = tp.kb(e);
+        const bool phase_r = e < tp.nR;
+        const int cls = tile_class(qb, kb, L, p.w0);
+        if (!warp_wait<CLUSTER>(sfull, e & 1, abort_flag, p.dev_error, 0x331)) { ok = false; break; }
+        tc_fence_after();
+        float x[BN];
+        {
+            uint32_t t0[32], t1[32], t2[32], t3[32];  // four loads in flight, one wait
+            tmem_ld32(s_col, t0);
+            tmem_ld32(s_col + 32, t1);
+            tmem_ld32(s_col + 64, t2);
+            tmem_ld32(s_col + 96, t3);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                x[u] = __uint_as_float(t0[u]);
+                x[32 + u] = __uint_as_float(t1[u]);
+                x[64 + u] = __uint_as_float(t2[u]);
+                x[96 + u] = __uint_as_float(t3[u]);
+            }
+        }
+        const int j0 = kb * BN;
+        const bool need_mask = (j0 + BN - 1 > qb * BM) || (j0 + BN > L) || cls == CLS_BAND;
+        if (need_mask) {
+            const int dw = i - j0 - p.w0;  // pair (i, j0 + u) is local iff u > dw
+#pragma unroll
+            for (int u = 0; u < BN; ++u) {
+                const int j = j0 + u;
+                bool masked = (j > i) || (j >= L);
+                if (cls == CLS_BAND) masked = masked || (phase_r ? (u > dw) : (u <= dw));
+                if (masked) x[u] = -INFINITY;
+            }
+        }
+        float m4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int u = 4; u < BN; u += 8) {
+            m4[0] = fmax3(m4[0], x[u], x[u + 1]);
+            m4[1] = fmax3(m4[1], x[u + 2], x[u + 3]);
+            m4[2] = fmax3(m4[2], x[u + 4], x[u + 5]);
+            m4[3] = fmax3(m4[3], x[u + 6], x[u + 7]);
+        }
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        const float m_new = fmaxf(m_used, mt);
+        const bool resc = m_new > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (resc) {
+            alpha = ex2_approx(m_used - m_new);
+            m_used = m_new;
+            l *= alpha;
+        }
+        const float ms = m_used == -INFINITY ? 0.f : m_used;
+        // p = 2^(x * scale * log2(e) - m), two columns per packed instruction
+        const float2 sl = make_float2(sl2, sl2), nm = make_float2(-ms, -ms);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int u = 0; u < BN; u += 4) {
+            const float2 y0 = fma2(make_float2(x[u], x[u + 1]), sl, nm);
+            const float2 y1 = fma2(make_float2(x[u + 2], x[u + 3]), sl, nm);
+            const float2 p0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+            const float2 p1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+            acc0 = add2(acc0, p0);
+            acc1 = add2(acc1, p1);
+            pk[u >> 1] = pack_bf16x2(p0.x, p0.y);
+            pk[(u >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+        }
+        l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        if (e > 0) {
+            // previous P.V of this head finished: O is stable and P's columns are free
+            if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, 0x332)) { ok = false; break; }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t tt[32];
+                    tmem_ld32(o_col + cc * 32, tt);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) tt[u] = __float_as_uint(__uint_as_float(tt[u]) * alpha);
+                    tmem_st32(o_col + cc * 32, tt);
+                }
+            }
+        }
+#pragma unroll
+        for (int cc = 0; cc < BN / 64; ++cc) {
+            uint32_t tt[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) tt[u] = pk[cc * 32 + u];
+            tmem_st32(s_col + cc * 32, tt);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_p();
+    }
+    // epilogue: O / l -> bf16 -> out
+    if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, 0x333)) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16* orow = p.out + (((size_t)b * p.Hq + head) * (size_t)L + (size_t)i) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t tt[32];
+            tmem_ld32(o_col + cc * 32, tt);
+            tmem_wait_ld();
+            if (i < L) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(tt[q * 8 + 0]) * inv, __uint_as_float(tt[q * 8 + 1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(tt[q * 8 + 2]) * inv, __uint_as_float(tt[q * 8 + 3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(tt[q * 8 + 4]) * inv, __uint_as_float(tt[q * 8 + 5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(tt[q * 8 + 6]) * inv, __uint_as_float(tt[q * 8 + 7]) * inv);
+                    *reinterpret_cast<uint4*>(orow + cc * 32 + q * 8) = v;
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+// [planes][L rows][d] bf16, box 64 columns x box_rows rows x 1 plane, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, int d, int L, int nplanes, int box_rows);
+
+// Parameters shared by both kernels (G magic numbers, RoPE turns, output).
+TcParams make_params(const PrefillProblem& pp);
+
+// The CTA-pair kernel (d = 128, query heads per kv head a multiple of 4).
+cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace jl

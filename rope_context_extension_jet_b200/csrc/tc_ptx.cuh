@@ -129,8 +129,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return d;
 }
 
-// Packed two-lane fp32 arithmetic (add/mul/fma .f32x2, sm_100): both lanes in
-// one instruction, round-to-nearest like the scalar forms.
+// Packed two-lane fp32 arithmetic (fma/add .f32x2, sm_100): both lanes in one
+// instruction, round-to-nearest like the scalar forms.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
 {
     float2 d;
@@ -139,16 +139,6 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
 __device__ __forceinline__ float2 add2(float2 a, float2 b)
@@ -170,6 +160,63 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar)
                  : "memory");
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The cta_group::2 forms: one MMA spans the two CTAs of a cluster pair.  Rows
+// [0, 128) of A and of D live in CTA 0 (its shared memory / TMEM), rows
+// [128, 256) in CTA 1; B is split along N, the first N/2 columns from CTA 0's
+// shared memory and the rest from CTA 1's, at the same offsets.  Every tcgen05
+// instruction of a kernel that uses them carries cta_group::2.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on the mbarrier at `bar`'s offset in both CTAs of the pair once every
+// pair MMA issued so far by this thread completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((unsigned short)0x3)
+        : "memory");
+}
+// Arrive on this CTA's `bar` only.
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 //   bits [0,14) start address >> 4; [16,30) leading byte offset >> 4;
 //   [32,46) stride byte offset >> 4; [46,48) version = 1; [49,52) base offset = 0;
@@ -183,44 +230,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
     return d;
-}
-
-// The same descriptor split into 32-bit words so that only the start-address
-// field (low word, bits [0,14)) changes per MMA: hi holds SBO, version and
-// layout; lo = (addr >> 4) | (LBO >> 4) << 16.  Adding (bytes >> 4) to lo moves
-// the start address (no carry out of the 14-bit field for addresses < 256 KB).
-__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo)
-{
-    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
-}
-__host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo)
-{
-    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
-}
-
-// MMA with the descriptors given as 32-bit word pairs and a compile-time
-// accumulate flag (no predicate set-up per instruction).
-template <bool ACC>
-__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
-                                          uint32_t b_hi, uint32_t idesc)
-{
-    asm volatile(
-        "{\n\t.reg .b64 da, db;\n\t"
-        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, %6;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(ACC ? 1 : 0)
-        : "memory");
-}
-template <bool ACC>
-__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                                          uint32_t idesc)
-{
-    asm volatile(
-        "{\n\t.reg .b64 db;\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, %5;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(ACC ? 1 : 0)
-        : "memory");
 }
 
 // Instruction descriptor for kind::f16 with fp16 A/B and fp32 accumulator

@@ -84,6 +84,27 @@ def test_batch_and_theta():
                     index=26))
 
 
+# Four (or eight) query heads per kv head with d = 128 take the CTA-pair kernel:
+# the same edge cases again on that path.
+@pytest.mark.parametrize("L", RAGGED)
+def test_ragged_lengths_head_quads(L):
+    full_case(small(f"quad-ragged-L{L}", Hq=4, Hkv=1, L=L, w_pre=max(1, L // 3), w0=17, index=29))
+
+
+@pytest.mark.parametrize("w0", W0_EDGES)
+def test_window_edges_head_quads(w0):
+    full_case(small(f"quad-w0-{w0}", Hq=8, Hkv=2, L=300, w_pre=100, w0=w0, index=30))
+
+
+def test_batch_and_theta_head_quads():
+    full_case(small("quad-batch2-theta1e4", B=2, Hq=8, Hkv=2, L=700, w_pre=90, w0=133, theta=1e4,
+                    index=31))
+
+
+def test_outlier_keys_head_quads():
+    full_case(small("quad-outliers", Hq=4, Hkv=1, L=1000, w_pre=500, w0=128, outliers=0.01, index=32))
+
+
 def test_outlier_keys_small():
     full_case(small("outliers", L=1000, w_pre=500, w0=128, outliers=0.01, index=27))
 
