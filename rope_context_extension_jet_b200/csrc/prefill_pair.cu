@@ -39,7 +39,7 @@ namespace tc {
 namespace {
 
 constexpr int D = 128;
-constexpr int NS = 4;           // ring depth of the K and V halves
+constexpr int NS = 5;           // ring depth of the K and V halves
 constexpr int KROWS = BN / 2;   // keys of a K tile held by one CTA
 constexpr int NTHREADS = 512;
 
@@ -132,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int nR = tp.nR, NE = tp.count();
 
     if (warp < 4) {
-        regs_dec<56>();
+        regs_dec<48>();
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
@@ -249,7 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
         }
     } else if (warp < 8) {
-        regs_dec<88>();
+        regs_dec<80>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
@@ -292,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (lane == 0) mbar_arrive_cluster(lead(P_KREADY + s));
         }
     } else {
-        regs_inc<184>();
+        regs_inc<192>();
         // -------------------------------------------------------------- softmax (head hh)
         const int hh = (warp - 8) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
