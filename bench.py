@@ -397,6 +397,28 @@ def main():
     dec_gbs = whole_job_rate(kv_bytes, world, dec_ms * 1e-3) / 1e9
     dec_tok_s = whole_job_rate(wd.B * wd.steps, world, dec_ms * 1e-3)
 
+    # ---------------- the same kernel in plain-RoPE mode (w0 >= L: every pair
+    # local, one phase, no band tiles), outside the timed region: the cost of
+    # the bifocal routing against plain RoPE attention on the same inputs
+    wplain = wp.with_(w0=wp.L)
+
+    def plain_call():
+        jl.prefill(qd, kd, vd, outd, w0=wplain.w0, w_pretrained=wplain.w_pretrained,
+                   rope_theta=wplain.rope_theta, scale=wplain.scale, stream=stream)
+
+    plain_call()
+    pl_ev = []
+    for _ in range(2):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plain_call()
+        b.record(stream)
+        pl_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    jl.device_status(stream)
+    plain_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in pl_ev])))
+    _, plain_computed, _, _ = prefill_flops(wplain)
+
     # ---------------- end to end through the public API with host buffers
     qh, kh, vh = to_pinned(q), to_pinned(k), to_pinned(v)
     outh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
@@ -435,7 +457,11 @@ def main():
                         "tiles": tiles, "band_tiles": band,
                         "tokens_per_s": round(world * wp.B * wp.L / (pre_ms * 1e-3), 1),
                         "frac_of_sustained_bf16": round(frac_s, 4),
-                        "frac_of_burst_bf16": round(pre_tflops / world / peaks["bf16_tflops"], 4)},
+                        "frac_of_burst_bf16": round(pre_tflops / world / peaks["bf16_tflops"], 4),
+                        "plain_rope_same_kernel": {
+                            "w0": wplain.w0, "ms": round(plain_ms, 3),
+                            "tflops_computed": round(whole_job_rate(plain_computed, world, plain_ms * 1e-3) / 1e12, 2),
+                            "bifocal_over_plain_time": round(pre_ms / plain_ms, 4)}},
             "decode": {"ms_per_token_step": round(dec_ms / wd.steps, 4),
                        "gbs_kv": round(dec_gbs, 1), "bytes_per_pass_kv": kv_bytes,
                        "bytes_per_pass_all": all_bytes, "tokens_per_s": round(dec_tok_s, 1),

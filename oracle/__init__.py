@@ -69,9 +69,11 @@ def load(path: str | None = None):
         lib.jlo_prefill_rows.restype = i32
         lib.jlo_prefill_rows.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                          dbl, dbl, vp, i64, vp, i32]
-        lib.jlo_decode.restype = i32
-        lib.jlo_decode.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32,
-                                   dbl, dbl, vp, i32]
+        for fn in (lib.jlo_decode, lib.jlo_decode_rope_cache):
+            fn.restype = i32
+            fn.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, dbl, dbl, vp, i32]
+        lib.jlo_rotate_rows.restype = i32
+        lib.jlo_rotate_rows.argtypes = [vp, i32, i64, i64, i32, dbl, vp]
         if path is None:
             _lib = lib
         return lib
@@ -143,7 +145,30 @@ def prefill(q, k, v, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=Non
     return out.reshape(B, Hq, L, d)
 
 
-def decode(q, kcache, vcache, L, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=None):
+def rotate_rows(x, rope_theta, lib=None) -> np.ndarray:
+    """Row j of every [rows, d] plane of x rotated to position j (fp64): a
+    standard RoPE key cache built from raw keys."""
+    x, dx = _as_input(x)
+    d, nrows = x.shape[-1], x.shape[-2]
+    nplanes = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    out = np.empty(x.shape, dtype=np.float64)
+    st = (lib or load()).jlo_rotate_rows(x.ctypes.data, dx, nplanes, nrows, d, float(rope_theta),
+                                         out.ctypes.data)
+    if st != 0:
+        raise ValueError(f"oracle rotate_rows failed with status {st}")
+    return out
+
+
+def decode_rope_cache(q, kcache, vcache, L, *, w0, w_pretrained, rope_theta, scale, nthreads=0,
+                      lib=None):
+    """Decode output [B,Hq,d] (fp64) over a standard RoPE cache: key row j is
+    stored rotated to its exact position j."""
+    return decode(q, kcache, vcache, L, w0=w0, w_pretrained=w_pretrained, rope_theta=rope_theta,
+                  scale=scale, nthreads=nthreads, lib=lib, _fn="jlo_decode_rope_cache")
+
+
+def decode(q, kcache, vcache, L, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=None,
+           _fn="jlo_decode"):
     """Decode output [B,Hq,d] (fp64) for a query at position L-1 over cache rows [0, L)."""
     q, dq = _as_input(q)
     kcache, dk = _as_input(kcache)
@@ -153,7 +178,7 @@ def decode(q, kcache, vcache, L, *, w0, w_pretrained, rope_theta, scale, nthread
     B, Hq, d = q.shape
     Hkv, Lcap = kcache.shape[1], kcache.shape[2]
     out = np.empty((B, Hq, d), dtype=np.float64)
-    st = (lib or load()).jlo_decode(q.ctypes.data, kcache.ctypes.data, vcache.ctypes.data, dq,
+    st = getattr(lib or load(), _fn)(q.ctypes.data, kcache.ctypes.data, vcache.ctypes.data, dq,
                                     B, Hq, Hkv, int(L), Lcap, d, int(w0), int(w_pretrained),
                                     float(rope_theta), float(scale), out.ctypes.data, int(nthreads))
     if st != 0:

@@ -115,6 +115,9 @@ typedef struct {
     /* cos/sin cache for positions [0, npos): cs[(p * h + m) * 2 + {0,1}] */
     const double* cs;
     int64_t npos;
+    /* 1: key rows are stored already rotated to their exact positions j (a
+     * standard RoPE cache); 0: raw key rows */
+    int rope_cache;
 } row_ctx;
 
 static void rotate_cached(const row_ctx* c, const double* x, double* y, int64_t p)
@@ -126,6 +129,20 @@ static void rotate_cached(const row_ctx* c, const double* x, double* y, int64_t 
         double a = x[m], b = x[m + h];
         y[m] = a * cc - b * ss;
         y[m + h] = a * ss + b * cc;
+    }
+}
+
+/* Rotation by -p (the inverse of the rotation to p): cos(-a) = cos a,
+ * sin(-a) = -sin a. */
+static void unrotate_cached(const row_ctx* c, const double* x, double* y, int64_t p)
+{
+    int h = c->d / 2;
+    const double* t = c->cs + (size_t)p * h * 2;
+    for (int m = 0; m < h; ++m) {
+        double cc = t[2 * m], ss = t[2 * m + 1];
+        double a = x[m], b = x[m + h];
+        y[m] = a * cc + b * ss;
+        y[m + h] = -a * ss + b * cc;
     }
 }
 
@@ -147,10 +164,15 @@ static void attend_row(const row_ctx* c, const void* q, size_t q_off,
         for (int t = 0; t < d; ++t) kraw[t] = widen(kbase, c->in_dtype, off + t);
         const double* qq;
         if (i - j < (int64_t)c->w0) {                  /* local branch  */
-            rotate_cached(c, kraw, kr, j);
+            if (c->rope_cache) memcpy(kr, kraw, sizeof(double) * (size_t)d);  /* already at j */
+            else rotate_cached(c, kraw, kr, j);
             qq = qe;
         } else {                                       /* remote branch */
-            rotate_cached(c, kraw, kr, jlo_remote_position(j, c->G));
+            int64_t fj = jlo_remote_position(j, c->G);
+            /* a key stored at j moves to f(j) by the extra rotation
+             * f(j) - j <= 0 (rotations compose additively) */
+            if (c->rope_cache) unrotate_cached(c, kraw, kr, j - fj);
+            else rotate_cached(c, kraw, kr, fj);
             qq = qm;
         }
         double a = 0.0;
@@ -271,11 +293,53 @@ int jlo_prefill_rows(const void* q, const void* k, const void* v, int in_dtype,
     return st;
 }
 
+static int decode_impl(const void* q, const void* kcache, const void* vcache, int in_dtype,
+                       int B, int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                       double rope_theta, double scale, double* out, int nthreads, int rope_cache);
+
 /* Decode: one new query per (b, h) at position i = L - 1 attending keys
- * [0, L) of caches [B,Hkv,Lcap,d]; G from this L.  out is [B,Hq,d]. */
+ * [0, L) of caches [B,Hkv,Lcap,d] holding raw key rows; G from this L.
+ * out is [B,Hq,d]. */
 int jlo_decode(const void* q, const void* kcache, const void* vcache, int in_dtype,
                int B, int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
                double rope_theta, double scale, double* out, int nthreads)
+{
+    return decode_impl(q, kcache, vcache, in_dtype, B, Hq, Hkv, L, Lcap, d, w0, w_pretrained,
+                       rope_theta, scale, out, nthreads, 0);
+}
+
+/* The same decode over a standard RoPE cache: row j of kcache holds the key
+ * already rotated to its exact position j.  Page 1, Metodologia 2: the cache
+ * keeps the base rotation; a remote key is moved to f(j) by the rotation
+ * f(j) - j (rotations compose additively), a local key is used as stored. */
+int jlo_decode_rope_cache(const void* q, const void* kcache, const void* vcache, int in_dtype,
+                          int B, int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                          double rope_theta, double scale, double* out, int nthreads)
+{
+    return decode_impl(q, kcache, vcache, in_dtype, B, Hq, Hkv, L, Lcap, d, w0, w_pretrained,
+                       rope_theta, scale, out, nthreads, 1);
+}
+
+/* Rotate every row j of x [nplanes][nrows][d] to position j (fp64 out):
+ * builds a standard RoPE key cache from raw keys. */
+int jlo_rotate_rows(const void* x, int in_dtype, int64_t nplanes, int64_t nrows, int d,
+                    double rope_theta, double* out)
+{
+    if (nplanes < 1 || nrows < 1 || d < 2 || d > 512 || (d & 1) || !(rope_theta > 0.0)) return -1;
+    if (in_dtype != JLO_IN_BF16 && in_dtype != JLO_IN_FP32) return -1;
+    double xr[512];
+    for (int64_t pl = 0; pl < nplanes; ++pl)
+        for (int64_t j = 0; j < nrows; ++j) {
+            size_t off = ((size_t)pl * (size_t)nrows + (size_t)j) * (size_t)d;
+            for (int t = 0; t < d; ++t) xr[t] = widen(x, in_dtype, off + (size_t)t);
+            jlo_rotate(xr, out + off, d, j, rope_theta);
+        }
+    return 0;
+}
+
+static int decode_impl(const void* q, const void* kcache, const void* vcache, int in_dtype,
+                       int B, int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                       double rope_theta, double scale, double* out, int nthreads, int rope_cache)
 {
     if (check_common(B, Hq, Hkv, L, d, w0, w_pretrained, rope_theta, in_dtype)) return -1;
     if (Lcap < L) return -1;
@@ -290,7 +354,7 @@ int jlo_decode(const void* q, const void* kcache, const void* vcache, int in_dty
     job_t J;
     memset(&J, 0, sizeof J);
     J.c.d = d; J.c.w0 = w0; J.c.G = jlo_group_size(L, w_pretrained);
-    J.c.scale = scale; J.c.in_dtype = in_dtype; J.c.npos = L;
+    J.c.scale = scale; J.c.in_dtype = in_dtype; J.c.npos = L; J.c.rope_cache = rope_cache;
     J.c.cs = build_cs(d, L, rope_theta);
     if (!J.c.cs) { free(rows); return -2; }
     J.q = q; J.k = kcache; J.v = vcache; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.L = L; J.Lkv = Lcap;

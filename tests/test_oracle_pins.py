@@ -3,7 +3,8 @@
 Each test ties the oracle to something other than itself: hand-evaluated values
 of G, Python's floor division, closed-form rotations, RoPE's relative-position
 property, textbook numpy RoPE attention in the cases the pages say reduce to it,
-and the pages' inclusion-exclusion formulation.  The mutation tests at the end
+the pages' inclusion-exclusion formulation, and (for decode over a standard
+RoPE cache) complex-number RoPE and the composition of rotations.  The mutation tests at the end
 plant plausible mistakes in copies of the oracle source and check that the pins
 catch every one of them.
 
@@ -199,10 +200,68 @@ def pin_decode_matches_prefill_row(lib):
     np.testing.assert_allclose(dec[0], pre, rtol=0, atol=1e-13)
 
 
+def pin_rotate_rows_textbook(lib):
+    # a standard RoPE cache built by the oracle equals the complex-number RoPE
+    x = _rand((2, 37, 16), 31)
+    got = oracle.rotate_rows(x, 1e4, lib=lib)
+    ref = tb.rope_complex(x.astype(np.float64), np.arange(37), 1e4)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def _decode_case(L, Hq=4, Hkv=2, d=16, seed=40):
+    q = _rand((1, Hq, d), seed)
+    k = _rand((1, Hkv, L + 3, d), seed + 1)
+    v = _rand((1, Hkv, L + 3, d), seed + 2)
+    return q, k, v
+
+
+def pin_rope_cache_decode_textbook(lib):
+    # Decode over a standard RoPE cache (key row j stored rotated to j) against
+    # textbook attention with the stored rows taken as they are: every pair
+    # local (w0 >= L) -> query at i, keys as stored; every pair remote (w0 = 0)
+    # -> query at f(i), stored key j moved by f(j) - j (complex RoPE handles the
+    # negative angle).  The stored rows are arbitrary vectors here.
+    L, sc, theta = 41, 0.3, 1e4
+    q, kc, vc = _decode_case(L)
+    group = 2
+    i = L - 1
+    for w0, w_pre in ((L, 9), (0, 9), (0, 41)):
+        G = -(-L // w_pre)
+        got = oracle.decode_rope_cache(q, kc, vc, L, w0=w0, w_pretrained=w_pre, rope_theta=theta,
+                                       scale=sc, lib=lib)
+        for h in range(q.shape[1]):
+            kk = kc[0, h // group, :L].astype(np.float64)
+            vv = vc[0, h // group, :L].astype(np.float64)
+            if w0 >= L:
+                qq = tb.rope_complex(q[0, h][None].astype(np.float64), np.array([i]), theta)
+                keys = kk
+            else:
+                qq = tb.rope_complex(q[0, h][None].astype(np.float64), np.array([i // G]), theta)
+                j = np.arange(L)
+                keys = tb.rope_complex(kk, j // G - j, theta)
+            ref, _ = tb.masked_attention(qq, keys, vv, sc, np.ones((1, L), bool))
+            np.testing.assert_allclose(got[0, h], ref[0], rtol=0, atol=1e-10)
+
+
+def pin_rope_cache_decode_composition(lib):
+    # Rotations compose: decoding a RoPE cache built from raw keys equals
+    # decoding the raw keys, for every window / group size (the cache is
+    # rounded to fp32, hence the tolerance).
+    L, sc, theta = 53, 0.25, 1e4
+    q, k, v = _decode_case(L, seed=50)
+    cache = tb.rope_complex(k.astype(np.float64), np.arange(k.shape[2]), theta).astype(np.float32)
+    for w0, w_pre in ((5, 9), (0, 20), (17, 5), (60, 7), (1, 53)):
+        kw = dict(w0=w0, w_pretrained=w_pre, rope_theta=theta, scale=sc, lib=lib)
+        a = oracle.decode_rope_cache(q, cache, v, L, **kw)
+        b = oracle.decode(q, k, v, L, **kw)
+        np.testing.assert_allclose(a, b, rtol=0, atol=2e-5)
+
+
 PINS = [pin_group_size_table, pin_remote_position, pin_rotation_closed_form,
         pin_rotation_algebra, pin_relative_invariance, pin_routing_enumeration,
         pin_reduction_g1, pin_reduction_wide_window, pin_reduction_zero_window,
-        pin_inclusion_exclusion, pin_decode_matches_prefill_row]
+        pin_inclusion_exclusion, pin_decode_matches_prefill_row, pin_rotate_rows_textbook,
+        pin_rope_cache_decode_textbook, pin_rope_cache_decode_composition]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -240,8 +299,7 @@ MUTANTS = {
     "window_boundary_le": ("if (i - j < (int64_t)c->w0) {", "if (i - j <= (int64_t)c->w0) {"),
     "query_not_aliased": ("rotate_cached(c, qraw, qm, jlo_remote_position(i, c->G));",
                           "rotate_cached(c, qraw, qm, i);"),
-    "key_not_aliased": ("rotate_cached(c, kraw, kr, jlo_remote_position(j, c->G));",
-                        "rotate_cached(c, kraw, kr, j);"),
+    "key_not_aliased": ("else rotate_cached(c, kraw, kr, fj);", "else rotate_cached(c, kraw, kr, j);"),
     "rotation_sign": ("y[m + h] = a * ss + b * cc;", "y[m + h] = -a * ss + b * cc;"),
     "interleaved_pairing": ("double a = x[m], b = x[m + h];\n        y[m] = a * cc - b * ss;\n"
                             "        y[m + h] = a * ss + b * cc;",
@@ -250,6 +308,12 @@ MUTANTS = {
     "frequency_exponent": ("return pow(rope_theta, -2.0 * (double)m / (double)d);",
                            "return pow(rope_theta, -1.0 * (double)m / (double)d);"),
     "gqa_modulo": ("int kvh = h / group;", "int kvh = h % J->Hkv;"),
+    "rope_cache_delta_sign": ("y[m] = a * cc + b * ss;\n        y[m + h] = -a * ss + b * cc;",
+                              "y[m] = a * cc - b * ss;\n        y[m + h] = a * ss + b * cc;"),
+    "rope_cache_local_rotated_again": ("if (c->rope_cache) memcpy(kr, kraw, sizeof(double) * (size_t)d);",
+                                       "if (c->rope_cache) rotate_cached(c, kraw, kr, j);"),
+    "rope_cache_moved_to_fj": ("if (c->rope_cache) unrotate_cached(c, kraw, kr, j - fj);",
+                               "if (c->rope_cache) rotate_cached(c, kraw, kr, fj);"),
     "dropped_self_key": ("for (int64_t j = 0; j <= i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
                          "        for (int t = 0; t < d; ++t) kraw[t]",
                          "for (int64_t j = 0; j < i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
