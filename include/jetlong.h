@@ -98,6 +98,22 @@ int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* 
                    jetlong_dtype dtype, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/* Decode over a standard RoPE key cache (the pages' own decode mechanism,
+ * Metodologia 2: the cache keeps every key at its base rotation and the
+ * bifocal positions are reached by correcting rotations, since rotations
+ * compose additively).  Row j of kcache holds the key already rotated to its
+ * exact position j, as an ordinary RoPE model writes it; vcache is unchanged.
+ * A local key (i - j < w0) is used as stored, a remote key is rotated by
+ * f(j) - j (<= 0) to reach f(j); the query is rotated to i or f(i) as in
+ * jetlong_decode.  Same arguments, sizes, workspace, ownership and errors as
+ * jetlong_decode; the result equals jetlong_decode on the raw keys up to the
+ * rounding of the stored rotated keys. */
+int jetlong_decode_rope_cache(const void* q, const void* kcache, const void* vcache, void* out,
+                              int B, int Hq, int Hkv, int L, int Lcap, int d,
+                              int w0, int w_pretrained, double rope_theta, float scale,
+                              jetlong_dtype dtype, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Allocation-free decode.  The paper has no counterpart to this entry point:
  * it exists for callers that cannot allocate device memory at all (a serving
  * runtime whose caching allocator must not grow, code running in a host

@@ -327,13 +327,21 @@ int jlo_rotate_rows(const void* x, int in_dtype, int64_t nplanes, int64_t nrows,
 {
     if (nplanes < 1 || nrows < 1 || d < 2 || d > 512 || (d & 1) || !(rope_theta > 0.0)) return -1;
     if (in_dtype != JLO_IN_BF16 && in_dtype != JLO_IN_FP32) return -1;
+    /* per-position cos/sin, computed once (the same libm values as jlo_rotate) */
+    row_ctx c;
+    memset(&c, 0, sizeof c);
+    c.d = d;
+    c.npos = nrows;
+    c.cs = build_cs(d, nrows, rope_theta);
+    if (!c.cs) return -2;
     double xr[512];
     for (int64_t pl = 0; pl < nplanes; ++pl)
         for (int64_t j = 0; j < nrows; ++j) {
             size_t off = ((size_t)pl * (size_t)nrows + (size_t)j) * (size_t)d;
             for (int t = 0; t < d; ++t) xr[t] = widen(x, in_dtype, off + (size_t)t);
-            jlo_rotate(xr, out + off, d, j, rope_theta);
+            rotate_cached(&c, xr, out + off, j);
         }
+    free((void*)c.cs);
     return 0;
 }
 

@@ -64,9 +64,10 @@ def load_library(path: str | None = None):
                                         dbl, flt, i32, vp]
         lib.jetlong_decode_workspace_size.restype = sz
         lib.jetlong_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
-        lib.jetlong_decode.restype = i32
-        lib.jetlong_decode.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
-                                       dbl, flt, i32, vp, sz, vp]
+        for fn in (lib.jetlong_decode, lib.jetlong_decode_rope_cache):
+            fn.restype = i32
+            fn.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                           dbl, flt, i32, vp, sz, vp]
         lib.jetlong_decode_noalloc.restype = i32
         lib.jetlong_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                                i32, dbl, flt, i32, vp]
@@ -160,8 +161,18 @@ def decode_workspace_size(B: int, Hq: int, Hkv: int, Lcap: int, d: int) -> int:
     return int(load_library().jetlong_decode_workspace_size(B, Hq, Hkv, Lcap, d))
 
 
+def decode_rope_cache(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
+                      rope_theta: float, scale: float | None = None, workspace=None, stream=None):
+    """One decode step over a standard RoPE cache (key row j stored rotated to
+    position j): jetlong_decode_rope_cache."""
+    return decode(q, kcache, vcache, L, out, w0=w0, w_pretrained=w_pretrained,
+                  rope_theta=rope_theta, scale=scale, workspace=workspace, stream=stream,
+                  _entry="jetlong_decode_rope_cache")
+
+
 def decode(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
-           rope_theta: float, scale: float | None = None, workspace=None, stream=None):
+           rope_theta: float, scale: float | None = None, workspace=None, stream=None,
+           _entry: str = "jetlong_decode"):
     """One decode step: raw q [B,Hq,d] at position L-1 over cache rows [0, L)."""
     import torch
     B, Hq, d = q.shape
@@ -175,7 +186,7 @@ def decode(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
-    _check(lib.jetlong_decode(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
+    _check(getattr(lib, _entry)(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
                               _dev(out, "out"), B, Hq, Hkv, int(L), Lcap, d, int(w0),
                               int(w_pretrained), float(rope_theta), float(scale),
                               _dtype_code(q), _dev(workspace, "workspace"),

@@ -291,7 +291,10 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
                             qhi[hh][u] = sq[(ver * HPB + hh) * D + H + m0 + u];
                         }
                 }
-                const uint32_t pos = exact ? (uint32_t)j : div_g((uint32_t)j, dl);
+                // raw keys go to j or f(j); keys stored at j stay, or move by f(j) - j <= 0
+                const uint32_t fj = div_g((uint32_t)j, dl);
+                const uint32_t pos = p.rope_cache ? (exact ? 0u : (uint32_t)j - fj) : (exact ? (uint32_t)j : fj);
+                const float sgn = (p.rope_cache && !exact) ? -1.f : 1.f;
                 float klo[PPL], khi[PPL];
                 const T* krow = reinterpret_cast<const T*>(kst + r * ROWB);
                 VecLoad<T, PPL>::run(krow + m0, klo);
@@ -303,6 +306,7 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
                 for (int u = 0; u < PPL; ++u) {
                     float cs, sn;
                     rope_cs_fast(pos, whi[u], wlo[u], cs, sn);
+                    sn *= sgn;
                     const float rl = klo[u] * cs - khi[u] * sn;
                     const float rh = klo[u] * sn + khi[u] * cs;
 #pragma unroll
@@ -448,9 +452,11 @@ __device__ __forceinline__ uint32_t dec_sw(uint32_t tile, int key, int ch)
 }
 
 // S^T for the 16 keys of this warp's block: rotated K fragments times Q^T.
+// Keys of rows g and g + 8 are rotated by the angles of positions pa and pb
+// (by minus those angles when sgn = -1).
 template <int D>
 __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int kw, int lane, uint32_t pa, uint32_t pb,
-                                             const uint2* sturns, const uint32_t (&qb)[D / 16][2])
+                                             float sgn, const uint2* sturns, const uint32_t (&qb)[D / 16][2])
 {
     const int g = lane >> 2, t = lane & 3;
     c[0] = c[1] = c[2] = c[3] = 0.f;
@@ -471,6 +477,8 @@ __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int 
             float c0, s0, c1, s1;
             rope_cs_fast(pos, w0.x, w0.y, c0, s0);
             rope_cs_fast(pos, w1.x, w1.y, c1, s1);
+            s0 *= sgn;
+            s1 *= sgn;
             const float x0 = bf16_lo(lo[r]), x1 = bf16_hi(lo[r]);
             const float y0 = bf16_lo(hi[r]), y1 = bf16_hi(hi[r]);
             lo[r] = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
@@ -595,15 +603,21 @@ __global__ void __launch_bounds__(TC_NT, 2)
             const uint32_t ktile = smem_u32(ring + st * C::STAGE), vtile = ktile + C::TILE;
             const int jb = j_begin + c * TC_KROWS + kw;  // first key of this warp's block
             const int ja = jb + g, jc = jb + g + 8;     // the keys of rows g and g + 8
+            // raw keys go to j (local) or f(j) (remote); keys stored rotated to
+            // j stay (local) or move by f(j) - j <= 0 (remote)
+            const uint32_t ea = p.rope_cache ? 0u : (uint32_t)ja, ec = p.rope_cache ? 0u : (uint32_t)jc;
+            const uint32_t fa = div_g((uint32_t)ja, dl), fc = div_g((uint32_t)jc, dl);
+            const uint32_t ra = p.rope_cache ? (uint32_t)ja - fa : fa, rc = p.rope_cache ? (uint32_t)jc - fc : fc;
+            const float rsgn = p.rope_cache ? -1.f : 1.f;
             float sc[4];
             if (jb >= j_exact) {
-                block_logits<D>(sc, ktile, kw, lane, (uint32_t)ja, (uint32_t)jc, sturns, qb_ex);
+                block_logits<D>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex);
             } else if (jb + 15 < j_exact) {
-                block_logits<D>(sc, ktile, kw, lane, div_g((uint32_t)ja, dl), div_g((uint32_t)jc, dl), sturns, qb_rm);
+                block_logits<D>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm);
             } else {
                 float se[4];
-                block_logits<D>(sc, ktile, kw, lane, div_g((uint32_t)ja, dl), div_g((uint32_t)jc, dl), sturns, qb_rm);
-                block_logits<D>(se, ktile, kw, lane, (uint32_t)ja, (uint32_t)jc, sturns, qb_ex);
+                block_logits<D>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm);
+                block_logits<D>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex);
                 if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
                 if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
             }

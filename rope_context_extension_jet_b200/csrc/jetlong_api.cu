@@ -165,10 +165,10 @@ size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int Lcap, int d)
     return jl::decode_workspace_bytes(B, Hq, Hkv, Lcap, d);
 }
 
-int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* out, int B,
-                   int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
-                   double rope_theta, float scale, jetlong_dtype dtype, void* workspace,
-                   size_t workspace_bytes, void* stream)
+static int decode_entry(const void* q, const void* kcache, const void* vcache, void* out, int B,
+                        int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                        double rope_theta, float scale, jetlong_dtype dtype, void* workspace,
+                        size_t workspace_bytes, void* stream, int rope_cache)
 {
     if (!q || !kcache || !vcache || !out || !workspace)
         return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
@@ -194,6 +194,7 @@ int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* 
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.Lcap = Lcap; p.d = d;
     p.w0 = w0 > L ? L : w0;
     p.G = (int)jetlong_group_size(L, w_pretrained);
+    p.rope_cache = rope_cache;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.workspace = workspace;
@@ -204,6 +205,24 @@ int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* 
     g_launches += n;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+int jetlong_decode(const void* q, const void* kcache, const void* vcache, void* out, int B,
+                   int Hq, int Hkv, int L, int Lcap, int d, int w0, int w_pretrained,
+                   double rope_theta, float scale, jetlong_dtype dtype, void* workspace,
+                   size_t workspace_bytes, void* stream)
+{
+    return decode_entry(q, kcache, vcache, out, B, Hq, Hkv, L, Lcap, d, w0, w_pretrained, rope_theta,
+                        scale, dtype, workspace, workspace_bytes, stream, 0);
+}
+
+int jetlong_decode_rope_cache(const void* q, const void* kcache, const void* vcache, void* out,
+                              int B, int Hq, int Hkv, int L, int Lcap, int d, int w0,
+                              int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
+                              void* workspace, size_t workspace_bytes, void* stream)
+{
+    return decode_entry(q, kcache, vcache, out, B, Hq, Hkv, L, Lcap, d, w0, w_pretrained, rope_theta,
+                        scale, dtype, workspace, workspace_bytes, stream, 1);
 }
 
 int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* out,

@@ -101,6 +101,7 @@ struct DecodeProblem {
     void* out;
     int B, Hq, Hkv, L, Lcap, d, w0;
     int G;
+    int rope_cache;  // 0: raw key rows; 1: key row j stored rotated to its exact position j
     float scale_log2;
     RopeTurns turns;
     void* workspace;

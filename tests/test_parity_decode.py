@@ -117,3 +117,65 @@ def test_cache_rows_past_length_are_ignored(dtype):
     ref = oracle.decode(np.ascontiguousarray(qs[0]), kc, vc, L, w0=w.w0,
                         w_pretrained=w.w_pretrained, rope_theta=w.rope_theta, scale=w.scale)
     check_gate(to_host_f64(out), ref, dtype, "decode with NaN rows past L")
+
+
+# ---------------------------------------------------------------- standard RoPE cache
+# jetlong_decode_rope_cache: key row j is stored rotated to its exact position
+# j (built here by the oracle from the seeded raw keys, rounded to the input
+# dtype); the reference is the oracle's decode over the same stored rows.
+
+def rope_cache_of(kc, w):
+    rot = oracle.rotate_rows(kc, w.rope_theta)
+    return I.to_bf16_bits(rot.astype(np.float32)) if w.dtype == "bf16" else rot.astype(np.float32)
+
+
+def check_rope_cache_steps(w, steps):
+    import torch
+    qs, kc, vc = I.decode_inputs(w)
+    kr = rope_cache_of(kc, w)
+    krd, vcd = to_device(kr), to_device(vc)
+    ws = torch.empty(jl.decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lcap, w.d), dtype=torch.uint8,
+                     device="cuda")
+    for t in steps:
+        qd = to_device(np.ascontiguousarray(qs[t]))
+        out = torch.full_like(qd, float("nan"))
+        jl.decode_rope_cache(qd, krd, vcd, w.length_at(t), out, w0=w.w0, w_pretrained=w.w_pretrained,
+                             rope_theta=w.rope_theta, scale=w.scale, workspace=ws)
+        jl.device_status()
+        ref = oracle.decode_rope_cache(np.ascontiguousarray(qs[t]), kr, vc, w.length_at(t), w0=w.w0,
+                                       w_pretrained=w.w_pretrained, rope_theta=w.rope_theta,
+                                       scale=w.scale)
+        check_gate(to_host_f64(out), ref, w.dtype, f"{w.name} rope-cache step {t}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("L0,w0", [(0, 64), (31, 64), (700, 64), (2999, 64), (2100, 0), (2100, 5000),
+                                   (1500, 1)])
+def test_rope_cache_decode_small(dtype, L0, w0):
+    check_rope_cache_steps(small_decode(f"rc-{dtype}-L{L0 + 1}-w{w0}", dtype=dtype, L0=L0, w0=w0,
+                                        steps=1, index=47), [0])
+
+
+def test_rope_cache_decode_crosses_group_boundary():
+    w = small_decode("rc-cross", L0=2998, Lcap=3008, steps=4, w_pre=1000, w0=100, index=48)
+    check_rope_cache_steps(w, [0, 1, 2, 3])
+
+
+def test_rope_cache_decode_full_size_g4_to_g5():
+    """B=8, Hq=32, Hkv=8, d=128, cache 131136 rows stored rotated; steps 31 (G=4) and 32 (G=5)."""
+    check_rope_cache_steps(I.D, [31, 32])
+
+
+def test_rope_cache_decode_matches_raw_cache_decode():
+    # the same attention reached two ways on the GPU: raw keys rotated in the
+    # kernel, or stored rotated keys corrected by f(j) - j
+    import torch
+    w = small_decode("rc-vs-raw", L0=2500, w_pre=600, w0=300, steps=1, index=49)
+    qs, kc, vc = I.decode_inputs(w)
+    kr = rope_cache_of(kc, w)
+    qd = to_device(np.ascontiguousarray(qs[0]))
+    kw = dict(w0=w.w0, w_pretrained=w.w_pretrained, rope_theta=w.rope_theta, scale=w.scale)
+    a = jl.decode_rope_cache(qd, to_device(kr), to_device(vc), w.length_at(0), **kw)
+    b = jl.decode(qd, to_device(kc), to_device(vc), w.length_at(0), **kw)
+    torch.cuda.synchronize()
+    check_gate(to_host_f64(a), to_host_f64(b), "bf16", "rope-cache decode vs raw-cache decode")
