@@ -39,12 +39,13 @@ METRIC = "bifocal prefill TFLOP/s & % bf16 peak at L=128K; decode HBM GB/s"
 BM = BN = 128  # tile shape used to count computed FLOPs
 
 
-def tile_counts(L, w0, bm=BM, bn=BN):
-    """(causal tiles, band tiles) of the (query-block, key-block) grid."""
-    nqb = (L + bm - 1) // bm
+def tile_counts(L, w0, bm=BM, bn=BN, P=0):
+    """(causal tiles, band tiles) of the (query-block, key-block) grid; query rows
+    are positions [P, L) (P = 0: the whole sequence)."""
+    nqb = (L - P + bm - 1) // bm
     tiles = band = 0
     for qb in range(nqb):
-        i_lo, i_hi = qb * bm, min(qb * bm + bm - 1, L - 1)
+        i_lo, i_hi = P + qb * bm, min(P + qb * bm + bm - 1, L - 1)
         nkb = i_hi // bn + 1
         tiles += nkb
         for kb in range(nkb):
@@ -55,9 +56,10 @@ def tile_counts(L, w0, bm=BM, bn=BN):
     return tiles, band
 
 
-def prefill_flops(w):
-    useful = 4.0 * w.d * w.Hq * w.B * w.L * (w.L + 1) / 2
-    tiles, band = tile_counts(w.L, min(w.w0, w.L))
+def prefill_flops(w, P=0):
+    """(useful, computed) FLOPs of the query rows [P, L) of workload w."""
+    useful = 4.0 * w.d * w.Hq * w.B * (w.L * (w.L + 1) / 2 - P * (P + 1) / 2)
+    tiles, band = tile_counts(w.L, min(w.w0, w.L), P=P)
     computed = w.B * w.Hq * (tiles * 4.0 * w.d * BM * BN + band * 2.0 * w.d * BM * BN)
     return useful, computed, tiles, band
 
@@ -419,6 +421,31 @@ def main():
     plain_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in pl_ev])))
     _, plain_computed, _, _ = prefill_flops(wplain)
 
+    # ---------------- chunked prefill (jetlong_prefill_chunk): the last 8192 rows
+    # of the same 128K sequence as one chunk over the resident K/V, outside the
+    # timed region
+    P_ch = wp.L - 8192
+    q_ch = qd[:, :, P_ch:].contiguous()
+    out_ch = torch.empty_like(q_ch)
+
+    def chunk_call():
+        jl.prefill_chunk(q_ch, kd, vd, P_ch, out_ch, w0=wp.w0, w_pretrained=wp.w_pretrained,
+                         rope_theta=wp.rope_theta, scale=wp.scale, stream=stream)
+
+    chunk_call()
+    ch_ev = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        chunk_call()
+        b.record(stream)
+        ch_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    jl.device_status(stream)
+    ch_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ch_ev])))
+    _, ch_computed, _, _ = prefill_flops(wp, P=P_ch)
+    del q_ch, out_ch
+
     # ---------------- decode over a standard RoPE cache (jetlong_decode_rope_cache),
     # one pass of the same 64 steps outside the timed region; the kernel's work
     # does not depend on the cached values, so the resident cache bytes serve
@@ -478,6 +505,9 @@ def main():
                         "tokens_per_s": round(world * wp.B * wp.L / (pre_ms * 1e-3), 1),
                         "frac_of_sustained_bf16": round(frac_s, 4),
                         "frac_of_burst_bf16": round(pre_tflops / world / peaks["bf16_tflops"], 4),
+                        "chunk_last_8192_rows": {
+                            "P": P_ch, "C": wp.L - P_ch, "ms": round(ch_ms, 3),
+                            "tflops_computed": round(whole_job_rate(ch_computed, world, ch_ms * 1e-3) / 1e12, 2)},
                         "plain_rope_same_kernel": {
                             "w0": wplain.w0, "ms": round(plain_ms, 3),
                             "tflops_computed": round(whole_job_rate(plain_computed, world, plain_ms * 1e-3) / 1e12, 2),

@@ -78,6 +78,23 @@ int jetlong_prefill(const void* q, const void* k, const void* v, void* out,
                     int w0, int w_pretrained, double rope_theta, float scale,
                     jetlong_dtype dtype, void* stream);
 
+/* Chunked prefill: the C new query rows of a sequence at positions
+ * [P, P + C) attend keys [0, i] of a cache that already holds the previous P
+ * keys and the chunk's own C keys, with G from the total length L = P + C
+ * (Metodologia 1: G follows the current length; a prompt can be processed in
+ * chunks that cross multiples of w_pretrained).  Row i's result equals row i of
+ * jetlong_prefill over the whole length-L sequence.
+ *   q [B,Hq,C,d] raw queries of the chunk; out [B,Hq,C,d] written.
+ *   kcache/vcache [B,Hkv,Lcap,d] raw keys/values, rows [0, P + C) valid (the
+ *   caller writes the chunk's keys/values at rows [P, P + C) first); rows
+ *   >= P + C are never read into the result.
+ *   P >= 0, C >= 1, P + C <= Lcap; other arguments as jetlong_prefill
+ *   (jetlong_prefill is this call with P = 0, C = Lcap = L). */
+int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache, void* out,
+                          int B, int Hq, int Hkv, int P, int C, int Lcap, int d,
+                          int w0, int w_pretrained, double rope_theta, float scale,
+                          jetlong_dtype dtype, void* stream);
+
 /* Bytes of device workspace jetlong_decode needs for any L <= Lcap with these
  * sizes (partial softmax states of the key splits plus merge counters).
  * Returns 0 for invalid sizes. */

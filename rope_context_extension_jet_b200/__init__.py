@@ -62,6 +62,9 @@ def load_library(path: str | None = None):
         lib.jetlong_prefill.restype = i32
         lib.jetlong_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                         dbl, flt, i32, vp]
+        lib.jetlong_prefill_chunk.restype = i32
+        lib.jetlong_prefill_chunk.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                              i32, i32, dbl, flt, i32, vp]
         lib.jetlong_decode_workspace_size.restype = sz
         lib.jetlong_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         for fn in (lib.jetlong_decode, lib.jetlong_decode_rope_cache):
@@ -154,6 +157,28 @@ def prefill(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: float,
     _check(lib.jetlong_prefill(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
                                B, Hq, Hkv, L, d, int(w0), int(w_pretrained), float(rope_theta),
                                float(scale), _dtype_code(q), _stream(stream)), lib)
+    return out
+
+
+def prefill_chunk(q, kcache, vcache, P: int, out=None, *, w0: int, w_pretrained: int,
+                  rope_theta: float, scale: float | None = None, stream=None):
+    """Chunked prefill: raw queries q [B,Hq,C,d] at positions [P, P+C) over cache
+    rows [0, P+C) of kcache/vcache [B,Hkv,Lcap,d]; G from P + C."""
+    import torch
+    B, Hq, C, d = q.shape
+    _, Hkv, Lcap, _ = kcache.shape
+    if vcache.shape != kcache.shape or kcache.shape[0] != B or kcache.shape[3] != d:
+        raise ValueError("kcache and vcache must be [B, Hkv, Lcap, d] matching q")
+    if not (q.dtype == kcache.dtype == vcache.dtype):
+        raise TypeError("q and the caches must share a dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_prefill_chunk(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
+                                     _dev(out, "out"), B, Hq, Hkv, int(P), C, Lcap, d, int(w0),
+                                     int(w_pretrained), float(rope_theta), float(scale),
+                                     _dtype_code(q), _stream(stream)), lib)
     return out
 
 

@@ -127,23 +127,27 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
     return ok();
 }
 
-int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq,
-                    int Hkv, int L, int d, int w0, int w_pretrained, double rope_theta,
-                    float scale, jetlong_dtype dtype, void* stream)
+static int prefill_entry(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                         int Hkv, int P, int C, int Lcap, int d, int w0, int w_pretrained,
+                         double rope_theta, float scale, jetlong_dtype dtype, void* stream)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return fail(JETLONG_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-    if (L < 1) return fail(JETLONG_ERR_INVALID_ARG, "L must be >= 1 (got %d)", L);
+    if (P < 0 || C < 1 || Lcap < 1 || (int64_t)P + C > Lcap)
+        return fail(JETLONG_ERR_INVALID_ARG, "need P >= 0, C >= 1, P + C <= Lcap (P=%d C=%d Lcap=%d)", P,
+                    C, Lcap);
     int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
     if (st != JETLONG_OK) return st;
     cudaError_t e;
     int* derr = dev_error_word(&e);
     if (!derr) return fail(JETLONG_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
 
+    const int L = P + C;
     jl::PrefillProblem p{};
     p.q = q; p.k = k; p.v = v; p.out = out;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.d = d;
+    p.P = P; p.C = C; p.Lcap = Lcap;
     p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
     p.G = (int)jetlong_group_size(L, w_pretrained);
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -156,6 +160,23 @@ int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int 
     g_launches += n;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                    int Hkv, int L, int d, int w0, int w_pretrained, double rope_theta,
+                    float scale, jetlong_dtype dtype, void* stream)
+{
+    if (L < 1) return fail(JETLONG_ERR_INVALID_ARG, "L must be >= 1 (got %d)", L);
+    return prefill_entry(q, k, v, out, B, Hq, Hkv, 0, L, L, d, w0, w_pretrained, rope_theta, scale,
+                         dtype, stream);
+}
+
+int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache, void* out, int B,
+                          int Hq, int Hkv, int P, int C, int Lcap, int d, int w0, int w_pretrained,
+                          double rope_theta, float scale, jetlong_dtype dtype, void* stream)
+{
+    return prefill_entry(q, kcache, vcache, out, B, Hq, Hkv, P, C, Lcap, d, w0, w_pretrained,
+                         rope_theta, scale, dtype, stream);
 }
 
 size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int Lcap, int d)

@@ -109,7 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars[P_DRAIN], 1);
         *abort_flag = 0;
-        *plan = plan_tiles(qb, p.L, p.w0);
+        *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
         // after a bounded wait expired anywhere in the grid (error word set),
         // later pairs skip their work; CTA 0 decides for both
         if (leader) *skip_word = *reinterpret_cast<volatile int*>(p.dev_error) != 0;
@@ -254,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
-        const uint32_t i0 = (uint32_t)(qb * BM);
+        const uint32_t i0 = (uint32_t)(p.P + qb * BM);
         bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, 0x431);
         if (ok) {
             for (int h = 0; h < 2; ++h) {
@@ -316,9 +316,9 @@ cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
 {
     CUtensorMap tq, tk, tv;
     cudaError_t e;
-    if ((e = make_map(&tq, pp.q, D, pp.L, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, pp.k, D, pp.L, pp.B * pp.Hkv, KROWS)) != cudaSuccess) return e;
-    if ((e = make_map(&tv, pp.v, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    if ((e = make_map(&tq, pp.q, D, pp.C, pp.C, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, KROWS)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);
     constexpr int smem = PairSmem::TOTAL;
     if ((e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=

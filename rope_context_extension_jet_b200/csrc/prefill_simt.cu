@@ -1,4 +1,6 @@
-// prefill_simt.cu -- fp32 CUDA-core prefill of dynamic bifocal RoPE attention.
+// prefill_simt.cu -- fp32 CUDA-core prefill of dynamic bifocal RoPE attention
+// (whole sequences, or a chunk of query rows at positions [P, P + C) against
+// the keys [0, P + C) of a cache).
 //
 // The fp32 element type (and its 1e-4 accuracy bar) rules out the tensor-core
 // path (TF32 keeps 10 mantissa bits), so fp32 inputs run here: a tiled
@@ -41,25 +43,26 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
 
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    const int nqb = (p.L + BM - 1) / BM;
+    const int nqb = (p.C + BM - 1) / BM;
     const int qb = nqb - 1 - blockIdx.x;  // heaviest query blocks first
     const int h = blockIdx.y, b = blockIdx.z;
     const int kvh = h / (p.Hq / p.Hkv);
     const int G = p.G;
 
-    const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * (size_t)p.L * D;
-    const T* k = reinterpret_cast<const T*>(p.k) + ((size_t)b * p.Hkv + kvh) * (size_t)p.L * D;
-    const T* v = reinterpret_cast<const T*>(p.v) + ((size_t)b * p.Hkv + kvh) * (size_t)p.L * D;
-    T* out = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + h) * (size_t)p.L * D;
+    // query row i (position P + r of the chunk) is row i - P of q and out
+    const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * (size_t)p.C * D;
+    const T* k = reinterpret_cast<const T*>(p.k) + ((size_t)b * p.Hkv + kvh) * (size_t)p.Lcap * D;
+    const T* v = reinterpret_cast<const T*>(p.v) + ((size_t)b * p.Hkv + kvh) * (size_t)p.Lcap * D;
+    T* out = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + h) * (size_t)p.C * D;
 
     // Q tile, rotated at i and at floor(i/G), pre-scaled into base-2 logit units.
     for (int e = tid; e < BM * H; e += NT) {
         int r = e / H, m = e % H;
-        int i = qb * BM + r;
+        int i = p.P + qb * BM + r;
         float a = 0.f, bb = 0.f;
         if (i < p.L) {
-            a = load_elem(q + (size_t)i * D + m);
-            bb = load_elem(q + (size_t)i * D + m + H);
+            a = load_elem(q + (size_t)(i - p.P) * D + m);
+            bb = load_elem(q + (size_t)(i - p.P) * D + m + H);
         }
         float c, s;
         rope_cs_accurate((uint32_t)i, p.turns.hi[m], p.turns.lo[m], c, s);
@@ -80,8 +83,8 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
         for (int c = 0; c < CPT; ++c) o[a][c] = 0.f;
     }
 
-    const int i_lo = qb * BM;
-    const int i_hi = min(qb * BM + BM - 1, p.L - 1);
+    const int i_lo = p.P + qb * BM;
+    const int i_hi = min(i_lo + BM - 1, p.L - 1);
     const int nkb = i_hi / BN + 1;
     for (int kb = 0; kb < nkb; ++kb) {
         const int j_lo = kb * BN, j_hi = kb * BN + BN - 1;
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
         if (i >= p.L) continue;
         float inv = 1.f / lrow[a];
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) store_elem(out + (size_t)i * D + tx + 16 * c, o[a][c] * inv);
+        for (int c = 0; c < CPT; ++c) store_elem(out + (size_t)(i - p.P) * D + tx + 16 * c, o[a][c] * inv);
     }
 }
 
@@ -243,7 +246,7 @@ cudaError_t launch_typed(const PrefillProblem& p, cudaStream_t st)
     const int smem = SimtSmem<D>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((p.L + BM - 1) / BM, p.Hq, p.B);
+    dim3 grid((p.C + BM - 1) / BM, p.Hq, p.B);
     kern<<<grid, NT, smem, st>>>(p);
     return cudaGetLastError();
 }

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
-        *plan = plan_tiles(qb, p.L, p.w0);
+        *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
-        const uint32_t i0 = (uint32_t)(qb * BM);
+        const uint32_t i0 = (uint32_t)(p.P + qb * BM);
         bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, 0x321);
         if (ok) {
             for (int h = 0; h < NH; ++h) {
@@ -299,9 +299,9 @@ cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
 {
     CUtensorMap tq, tk, tv;
     cudaError_t e;
-    if ((e = make_map(&tq, pp.q, D, pp.L, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, pp.k, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
-    if ((e = make_map(&tv, pp.v, D, pp.L, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    if ((e = make_map(&tq, pp.q, D, pp.C, pp.C, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);
     auto kern = prefill_tc_kernel<D, NH>;
     constexpr int smem = TcSmem<D, NH>::TOTAL;
@@ -344,13 +344,14 @@ void make_div_magic(uint32_t G, uint32_t* m, uint32_t* s1, uint32_t* s2)
 
 }  // namespace
 
-cudaError_t make_map(CUtensorMap* m, const void* base, int d, int L, int nplanes, int box_rows)
+cudaError_t make_map(CUtensorMap* m, const void* base, int d, int rows, int plane_rows, int nplanes,
+                     int box_rows)
 {
     cudaError_t err;
     EncodeTiledFn fn = encode_fn(&err);
     if (!fn) return err == cudaSuccess ? cudaErrorSymbolNotFound : err;
-    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)nplanes};
-    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)nplanes};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)plane_rows * d * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -363,7 +364,8 @@ TcParams make_params(const PrefillProblem& pp)
 {
     TcParams p{};
     p.B = pp.B; p.Hq = pp.Hq; p.Hkv = pp.Hkv; p.L = pp.L; p.w0 = pp.w0; p.G = pp.G;
-    p.nqb = (pp.L + BM - 1) / BM;
+    p.P = pp.P; p.C = pp.C;
+    p.nqb = (pp.C + BM - 1) / BM;
     make_div_magic((uint32_t)pp.G, &p.div_m, &p.div_s1, &p.div_s2);
     p.scale_log2 = pp.scale_log2;
     p.turns = pp.turns;

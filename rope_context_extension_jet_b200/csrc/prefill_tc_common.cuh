@@ -28,8 +28,11 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when th
 
 enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
 
+// Query rows are positions [P, P + C) (row i of q / out is position P + i),
+// keys [0, L), L = P + C; nqb query blocks of BM rows.
 struct TcParams {
     int B, Hq, Hkv, L, w0, G, nqb;
+    int P, C;
     uint32_t div_m, div_s1, div_s2;  // floor(x / G) by multiply-shift
     float scale_log2;
     RopeTurns turns;
@@ -45,11 +48,11 @@ __device__ __forceinline__ uint32_t div_g(uint32_t n, const TcParams& p)
     return (t1 + ((n - t1) >> p.div_s1)) >> p.div_s2;
 }
 
-// Class of the (query block qb, key block kb) tile: every pair local, every
-// pair remote, or both (the band i - j = w0 crosses the tile).
-__device__ __forceinline__ int tile_class(int qb, int kb, int L, int w0)
+// Class of the tile (query rows from position i_lo, key block kb): every pair
+// local, every pair remote, or both (the band i - j = w0 crosses the tile).
+__device__ __forceinline__ int tile_class(int i_lo, int kb, int L, int w0)
 {
-    const int i_lo = qb * BM, i_hi = min(qb * BM + BM - 1, L - 1);
+    const int i_hi = min(i_lo + BM - 1, L - 1);
     const int dmax = i_hi - kb * BN;
     const int dmin = max(0, i_lo - (kb * BN + BN - 1));
     if (dmax < w0) return CLS_LOC;
@@ -57,23 +60,24 @@ __device__ __forceinline__ int tile_class(int qb, int kb, int L, int w0)
     return CLS_BAND;
 }
 
-// Key tiles of query block qb in processing order: phase R = [0, nR) (remote
-// and band tiles, rotated at the aliased positions), then phase E = [kE0, nkb)
-// (band and local tiles, rotated at the exact positions).
+// Key tiles of the query block starting at position i_lo in processing order:
+// phase R = [0, nR) (remote and band tiles, rotated at the aliased positions),
+// then phase E = [kE0, nkb) (band and local tiles, rotated at the exact
+// positions).
 struct TilePlan {
     int nR, kE0, nkb;
     __device__ __forceinline__ int count() const { return nR + (nkb - kE0); }
     __device__ __forceinline__ int kb(int e) const { return e < nR ? e : kE0 + (e - nR); }
 };
 
-__device__ __forceinline__ TilePlan plan_tiles(int qb, int L, int w0)
+__device__ __forceinline__ TilePlan plan_tiles(int i_lo, int L, int w0)
 {
     TilePlan t;
-    t.nkb = min(qb * BM + BM - 1, L - 1) / BN + 1;
+    t.nkb = min(i_lo + BM - 1, L - 1) / BN + 1;
     t.nR = t.nkb;
     t.kE0 = t.nkb;
     for (int kb = 0; kb < t.nkb; ++kb) {
-        const int cls = tile_class(qb, kb, L, w0);
+        const int cls = tile_class(i_lo, kb, L, w0);
         if (cls != CLS_REM && t.kE0 == t.nkb) t.kE0 = kb;
         if (cls == CLS_LOC) { t.nR = kb; break; }
     }
@@ -207,7 +211,8 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
 {
     const int lane = r & 31;
     const int L = p.L;
-    const int i = qb * BM + r;
+    const int i_lo = p.P + qb * BM;
+    const int i = i_lo + r;
     const int NE = tp.count();
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
@@ -215,7 +220,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
     for (int e = 0; e < NE; ++e) {
         const int kb = tp.kb(e);
         const bool phase_r = e < tp.nR;
-        const int cls = tile_class(qb, kb, L, p.w0);
+        const int cls = tile_class(i_lo, kb, L, p.w0);
         if (!warp_wait<CLUSTER>(sfull, e & 1, abort_flag, p.dev_error, 0x331)) { ok = false; break; }
         tc_fence_after();
         float x[BN];
@@ -235,7 +240,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
             }
         }
         const int j0 = kb * BN;
-        const bool need_mask = (j0 + BN - 1 > qb * BM) || (j0 + BN > L) || cls == CLS_BAND;
+        const bool need_mask = (j0 + BN - 1 > i_lo) || (j0 + BN > L) || cls == CLS_BAND;
         if (need_mask) {
             const int dw = i - j0 - p.w0;  // pair (i, j0 + u) is local iff u > dw
 #pragma unroll
@@ -312,7 +317,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
     if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, 0x333)) {
         tc_fence_after();
         const float inv = 1.f / l;
-        __nv_bfloat16* orow = p.out + (((size_t)b * p.Hq + head) * (size_t)L + (size_t)i) * D;
+        __nv_bfloat16* orow = p.out + (((size_t)b * p.Hq + head) * (size_t)p.C + (size_t)(i - p.P)) * D;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t tt[32];
@@ -335,8 +340,10 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
 
 // ------------------------------------------------------------------ host side
 
-// [planes][L rows][d] bf16, box 64 columns x box_rows rows x 1 plane, 128-byte swizzle.
-cudaError_t make_map(CUtensorMap* m, const void* base, int d, int L, int nplanes, int box_rows);
+// [planes][plane_rows][d] bf16 read as rows [0, rows) of every plane (rows >=
+// rows load as zeros), box 64 columns x box_rows rows x 1 plane, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, int d, int rows, int plane_rows, int nplanes,
+                     int box_rows);
 
 // Parameters shared by both kernels (G magic numbers, RoPE turns, output).
 TcParams make_params(const PrefillProblem& pp);

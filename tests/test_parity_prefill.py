@@ -161,3 +161,88 @@ def test_position_map_bit_exact():
         np.testing.assert_array_equal(got, ref)
         full = out.cpu().numpy()
         np.testing.assert_array_equal(full, np.arange(L) // G)
+
+
+# ---------------------------------------------------------------- chunked prefill
+# jetlong_prefill_chunk: the C query rows at positions [P, P + C) over cache rows
+# [0, P + C); G from P + C.  Reference: the oracle's prefill rows i in [P, P + C)
+# of the length-(P + C) sequence made of the same cache rows.
+
+def chunk_case(name, P, C, Lcap, *, dtype="bf16", B=1, Hq=4, Hkv=1, d=128, w_pre=100, w0=17,
+               theta=1e6, index=60, nan_tail=False, rows=None):
+    import torch
+    L = P + C
+    w = I.PrefillWorkload(name, index, dtype, B, Hq, Hkv, d, Lcap, w_pre, w0, theta)
+    q, k, v = I.prefill_inputs(w)
+    qc = np.ascontiguousarray(q[:, :, P:L])
+    kd, vd = to_device(k), to_device(v)
+    if nan_tail and L < Lcap:
+        kd[:, :, L:] = float("nan")
+        vd[:, :, L:] = float("nan")
+    out = torch.full_like(to_device(qc), float("nan"))
+    jl.prefill_chunk(to_device(qc), kd, vd, P, out, w0=w0, w_pretrained=w_pre, rope_theta=theta,
+                     scale=w.scale)
+    jl.device_status()
+    got = to_host_f64(out)
+    if rows is None:
+        bb, hh, ii = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(P, L), indexing="ij")
+        rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
+    rows = np.asarray(rows, dtype=np.int32)
+    ref = oracle.prefill_rows(np.ascontiguousarray(q[:, :, :L]), np.ascontiguousarray(k[:, :, :L]),
+                              np.ascontiguousarray(v[:, :, :L]), rows, w0=w0, w_pretrained=w_pre,
+                              rope_theta=theta, scale=w.scale)
+    sel = got[rows[:, 0], rows[:, 1], rows[:, 2] - P]
+    return check_gate(sel, ref, dtype, name)
+
+
+CHUNKS = [(0, 300), (128, 256), (100, 77), (1000, 1), (999, 130), (300, 700), (5, 1200)]
+
+
+@pytest.mark.parametrize("P,C", CHUNKS)
+def test_chunk_head_quads(P, C):
+    chunk_case(f"chunk-q-{P}-{C}", P, C, P + C + 40, index=61)
+
+
+@pytest.mark.parametrize("P,C", [(128, 256), (100, 77), (999, 130)])
+def test_chunk_head_pairs_and_single(P, C):
+    chunk_case(f"chunk-p-{P}-{C}", P, C, P + C + 3, Hq=4, Hkv=2, index=62)
+    chunk_case(f"chunk-s-{P}-{C}", P, C, P + C + 3, Hq=3, Hkv=3, index=63)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("P,C", [(0, 200), (150, 90), (511, 1)])
+def test_chunk_fp32(d, P, C):
+    chunk_case(f"chunk-f32-{d}-{P}-{C}", P, C, P + C + 5, dtype="fp32", Hq=2, Hkv=1, d=d, index=64)
+
+
+@pytest.mark.parametrize("w0", [0, 1, 128, 5000])
+def test_chunk_windows(w0):
+    chunk_case(f"chunk-w0-{w0}", 700, 300, 1100, Hq=8, Hkv=2, w0=w0, w_pre=240, index=65)
+
+
+def test_chunk_ignores_cache_rows_past_length():
+    chunk_case("chunk-nan-tail", 600, 200, 1024, nan_tail=True, index=66)
+    chunk_case("chunk-nan-tail-f32", 600, 200, 1024, dtype="fp32", Hq=2, d=64, nan_tail=True, index=66)
+
+
+def test_chunk_of_one_row_equals_decode():
+    import torch
+    P, Lcap = 1536, 1600
+    w = I.PrefillWorkload("chunk-vs-decode", 67, "bf16", 2, 8, 2, 128, Lcap, 400, 200, 1e6)
+    q, k, v = I.prefill_inputs(w)
+    qd, kd, vd = to_device(q), to_device(k), to_device(v)
+    kw = dict(w0=w.w0, w_pretrained=w.w_pretrained, rope_theta=w.rope_theta, scale=w.scale)
+    ch = jl.prefill_chunk(qd[:, :, P:P + 1].contiguous(), kd, vd, P, **kw)
+    dec = jl.decode(qd[:, :, P].contiguous(), kd, vd, P + 1, **kw)
+    torch.cuda.synchronize()
+    check_gate(to_host_f64(ch[:, :, 0]), to_host_f64(dec), "bf16", "one-row chunk vs decode")
+
+
+def test_chunk_of_128k_sequence_sampled():
+    """The last 4096 rows of the 131072-token headline sequence as one chunk (G = 4)."""
+    P, C = 131072 - 4096, 4096
+    rng = np.random.default_rng(68)
+    rows = [(0, h, P + int(r)) for h in (0, 9, 22, 31) for r in
+            list(range(0, 8)) + list(range(C - 8, C)) + list(rng.integers(0, C, 8))]
+    chunk_case("chunk-128k", P, C, P + C, B=1, Hq=32, Hkv=8, d=128, w_pre=32768, w0=4096, index=69,
+               rows=rows)
