@@ -112,3 +112,40 @@ def test_position_map_rejects_bad_arguments(lib):
     assert lib.jetlong_position_map(NULL, 10, 4, NULL) == 1
     assert lib.jetlong_position_map(P, 0, 4, NULL) == 1
     assert lib.jetlong_position_map(P, 10, 0, NULL) == 1
+
+
+def _chunk(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, B=1, Hq=4, Hkv=1, P0=100, C=28, Lcap=128, d=128, w0=8, wp=32,
+             theta=1e6, scale=0.088, dtype=0)
+    a.update(kw)
+    return lib.jetlong_prefill_chunk(a["q"], a["kc"], a["vc"], a["out"], a["B"], a["Hq"], a["Hkv"],
+                                     a["P0"], a["C"], a["Lcap"], a["d"], a["w0"], a["wp"], a["theta"],
+                                     a["scale"], a["dtype"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=NULL), 1), (dict(vc=NULL), 1), (dict(P0=-1), 1), (dict(C=0), 1), (dict(C=29), 1),
+    (dict(Lcap=0), 1), (dict(Hkv=3), 1), (dict(d=96), 2), (dict(wp=0), 1), (dict(dtype=5), 1),
+    (dict(out=ctypes.c_void_p((1 << 20) + 8)), 1),
+])
+def test_prefill_chunk_rejects_bad_arguments_on_host(lib, kw, status):
+    before = jl.launch_count()
+    assert _chunk(lib, **kw) == status
+    assert jl.launch_count() == before
+    assert jl.last_error() != ""
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kc=NULL), 1), (dict(ws=NULL), 1), (dict(L=0), 1), (dict(L=129), 1), (dict(wsb=16), 1),
+    (dict(Hkv=3), 1), (dict(d=80), 2),
+])
+def test_decode_rope_cache_rejects_bad_arguments_on_host(lib, kw, status):
+    a = dict(q=P, kc=P, vc=P, out=P, B=2, Hq=8, Hkv=2, L=100, Lcap=128, d=128, w0=8, wp=32,
+             theta=1e6, scale=0.088, dtype=0, ws=P, wsb=1 << 30)
+    a.update(kw)
+    before = jl.launch_count()
+    st = lib.jetlong_decode_rope_cache(a["q"], a["kc"], a["vc"], a["out"], a["B"], a["Hq"], a["Hkv"],
+                                       a["L"], a["Lcap"], a["d"], a["w0"], a["wp"], a["theta"],
+                                       a["scale"], a["dtype"], a["ws"], a["wsb"], NULL)
+    assert st == status
+    assert jl.launch_count() == before
