@@ -69,6 +69,9 @@ def load(path: str | None = None):
         lib.jlo_prefill_rows.restype = i32
         lib.jlo_prefill_rows.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                          dbl, dbl, vp, i64, vp, i32]
+        lib.jlo_prefill_rows_lse.restype = i32
+        lib.jlo_prefill_rows_lse.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                             dbl, dbl, vp, i64, vp, vp, i32]
         for fn in (lib.jlo_decode, lib.jlo_decode_rope_cache):
             fn.restype = i32
             fn.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, dbl, dbl, vp, i32]
@@ -111,8 +114,10 @@ def pair_logit(q, k, i, j, w0, G, rope_theta, lib=None) -> float:
                                                 int(i), int(j), int(w0), int(G), float(rope_theta)))
 
 
-def prefill_rows(q, k, v, rows, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=None):
-    """Routed attention outputs (fp64, [n, d]) for the (b, h, i) triples in ``rows``.
+def prefill_rows(q, k, v, rows, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=None,
+                 with_lse=False):
+    """Routed attention outputs (fp64, [n, d]) for the (b, h, i) triples in ``rows``
+    (and, with ``with_lse``, each row's log sum_j exp(scale * logit) as [n]).
 
     q: [B,Hq,L,d], k/v: [B,Hkv,L,d] as uint16 bf16 bits or float32.
     """
@@ -125,14 +130,15 @@ def prefill_rows(q, k, v, rows, *, w0, w_pretrained, rope_theta, scale, nthreads
     Hkv = k.shape[1]
     rows = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
     out = np.empty((rows.shape[0], d), dtype=np.float64)
-    st = (lib or load()).jlo_prefill_rows(q.ctypes.data, k.ctypes.data, v.ctypes.data, dq,
-                                          B, Hq, Hkv, L, d, int(w0), int(w_pretrained),
-                                          float(rope_theta), float(scale),
-                                          rows.ctypes.data, rows.shape[0], out.ctypes.data,
-                                          int(nthreads))
+    lse = np.empty(rows.shape[0], dtype=np.float64)
+    st = (lib or load()).jlo_prefill_rows_lse(q.ctypes.data, k.ctypes.data, v.ctypes.data, dq,
+                                              B, Hq, Hkv, L, d, int(w0), int(w_pretrained),
+                                              float(rope_theta), float(scale),
+                                              rows.ctypes.data, rows.shape[0], out.ctypes.data,
+                                              lse.ctypes.data, int(nthreads))
     if st != 0:
         raise ValueError(f"oracle prefill_rows failed with status {st}")
-    return out
+    return (out, lse) if with_lse else out
 
 
 def prefill(q, k, v, *, w0, w_pretrained, rope_theta, scale, nthreads=0, lib=None):

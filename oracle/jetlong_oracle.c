@@ -150,7 +150,7 @@ static void unrotate_cached(const row_ctx* c, const double* x, double* y, int64_
  * at element offset j * d.  Query position i, keys j in [0, i].          */
 static void attend_row(const row_ctx* c, const void* q, size_t q_off,
                        const void* kbase, const void* vbase, size_t kv_off,
-                       int64_t i, double* logit, double* out)
+                       int64_t i, double* logit, double* out, double* lse)
 {
     int d = c->d;
     double qraw[512], qe[512], qm[512], kraw[512], kr[512];
@@ -189,6 +189,8 @@ static void attend_row(const row_ctx* c, const void* q, size_t q_off,
         for (int t = 0; t < d; ++t) out[t] += p * widen(vbase, c->in_dtype, off + t);
     }
     for (int t = 0; t < d; ++t) out[t] /= sum;
+    /* log of the softmax denominator: log sum_j exp(scale * a_ij) */
+    if (lse) *lse = mx + log(sum);
 }
 
 static double* build_cs(int d, int64_t npos, double rope_theta)
@@ -216,6 +218,7 @@ typedef struct {
     const int32_t* rows;    /* n triples (b, h, i) */
     int64_t n;
     double* out;
+    double* lse;  /* optional: one log-sum-exp per row */
     int64_t next; /* work counter */
     int status;
 } job_t;
@@ -236,7 +239,8 @@ static void* worker(void* arg)
         size_t q_off = J->q_is_decode ? ((size_t)b * J->Hq + h) * d
                                       : (((size_t)b * J->Hq + h) * J->L + i) * d;
         size_t kv_off = ((size_t)b * J->Hkv + kvh) * (size_t)J->Lkv * d;
-        attend_row(&J->c, J->q, q_off, J->k, J->v, kv_off, i, logit, J->out + (size_t)r * d);
+        attend_row(&J->c, J->q, q_off, J->k, J->v, kv_off, i, logit, J->out + (size_t)r * d,
+                   J->lse ? J->lse + r : NULL);
     }
     free(logit);
     return NULL;
@@ -270,10 +274,26 @@ static int check_common(int B, int Hq, int Hkv, int L, int d, int w0, int w_pret
 /* Prefill rows: out[r, :] = routed attention output of query (b, h, i) for
  * the n triples in rows; q [B,Hq,L,d], k/v [B,Hkv,L,d], one G for the call
  * computed from L.  Returns 0 on success. */
+int jlo_prefill_rows_lse(const void* q, const void* k, const void* v, int in_dtype,
+                         int B, int Hq, int Hkv, int L, int d, int w0, int w_pretrained,
+                         double rope_theta, double scale,
+                         const int32_t* rows, int64_t n, double* out, double* lse, int nthreads);
+
 int jlo_prefill_rows(const void* q, const void* k, const void* v, int in_dtype,
                      int B, int Hq, int Hkv, int L, int d, int w0, int w_pretrained,
                      double rope_theta, double scale,
                      const int32_t* rows, int64_t n, double* out, int nthreads)
+{
+    return jlo_prefill_rows_lse(q, k, v, in_dtype, B, Hq, Hkv, L, d, w0, w_pretrained, rope_theta,
+                                scale, rows, n, out, NULL, nthreads);
+}
+
+/* The same rows plus lse[r] = log sum_j exp(scale * a_ij) of each row (the
+ * statistic the pages' inclusion-exclusion merge combines, Metodologia 2). */
+int jlo_prefill_rows_lse(const void* q, const void* k, const void* v, int in_dtype,
+                         int B, int Hq, int Hkv, int L, int d, int w0, int w_pretrained,
+                         double rope_theta, double scale,
+                         const int32_t* rows, int64_t n, double* out, double* lse, int nthreads)
 {
     if (check_common(B, Hq, Hkv, L, d, w0, w_pretrained, rope_theta, in_dtype)) return -1;
     for (int64_t r = 0; r < n; ++r)
@@ -287,7 +307,7 @@ int jlo_prefill_rows(const void* q, const void* k, const void* v, int in_dtype,
     J.c.cs = build_cs(d, L, rope_theta);
     if (!J.c.cs) return -2;
     J.q = q; J.k = k; J.v = v; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.L = L; J.Lkv = L;
-    J.rows = rows; J.n = n; J.out = out;
+    J.rows = rows; J.n = n; J.out = out; J.lse = lse;
     int st = run_job(&J, nthreads);
     free((void*)J.c.cs);
     return st;

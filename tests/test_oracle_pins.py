@@ -200,6 +200,24 @@ def pin_decode_matches_prefill_row(lib):
     np.testing.assert_allclose(dec[0], pre, rtol=0, atol=1e-13)
 
 
+def pin_row_lse_textbook(lib):
+    # each row's log-sum-exp equals textbook RoPE attention's, where the method
+    # reduces to it: G = 1 (any window), w0 >= L, and w0 = 0 at positions // G
+    L, Hq, Hkv, d, sc = 40, 4, 2, 16, 0.3
+    q = _rand((1, Hq, L, d), 61)
+    k = _rand((1, Hkv, L, d), 62)
+    v = _rand((1, Hkv, L, d), 63)
+    b, h, i = np.meshgrid(np.arange(1), np.arange(Hq), np.arange(L), indexing="ij")
+    rows = np.stack([b.ravel(), h.ravel(), i.ravel()], axis=1)
+    kk = tb.repeat_kv(k.astype(np.float64), Hq // Hkv)
+    vv = tb.repeat_kv(v.astype(np.float64), Hq // Hkv)
+    for w0, w_pre, pos in ((7, 64, np.arange(L)), (L, 9, np.arange(L)), (0, 9, np.arange(L) // 5)):
+        _, lse = oracle.prefill_rows(q, k, v, rows, w0=w0, w_pretrained=w_pre, rope_theta=1e4,
+                                     scale=sc, with_lse=True, lib=lib)
+        _, ref = tb.rope_attention(q.astype(np.float64), kk, vv, pos, 1e4, sc)
+        np.testing.assert_allclose(lse, ref.reshape(-1), rtol=0, atol=1e-10)
+
+
 def pin_rotate_rows_textbook(lib):
     # a standard RoPE cache built by the oracle equals the complex-number RoPE
     x = _rand((2, 37, 16), 31)
@@ -260,7 +278,8 @@ def pin_rope_cache_decode_composition(lib):
 PINS = [pin_group_size_table, pin_remote_position, pin_rotation_closed_form,
         pin_rotation_algebra, pin_relative_invariance, pin_routing_enumeration,
         pin_reduction_g1, pin_reduction_wide_window, pin_reduction_zero_window,
-        pin_inclusion_exclusion, pin_decode_matches_prefill_row, pin_rotate_rows_textbook,
+        pin_inclusion_exclusion, pin_decode_matches_prefill_row, pin_row_lse_textbook,
+        pin_rotate_rows_textbook,
         pin_rope_cache_decode_textbook, pin_rope_cache_decode_composition]
 
 
@@ -314,6 +333,7 @@ MUTANTS = {
                                        "if (c->rope_cache) rotate_cached(c, kraw, kr, j);"),
     "rope_cache_moved_to_fj": ("if (c->rope_cache) unrotate_cached(c, kraw, kr, j - fj);",
                                "if (c->rope_cache) rotate_cached(c, kraw, kr, fj);"),
+    "lse_without_max": ("if (lse) *lse = mx + log(sum);", "if (lse) *lse = log(sum);"),
     "dropped_self_key": ("for (int64_t j = 0; j <= i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
                          "        for (int t = 0; t < d; ++t) kraw[t]",
                          "for (int64_t j = 0; j < i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
