@@ -95,6 +95,21 @@ int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache,
                           int w0, int w_pretrained, double rope_theta, float scale,
                           jetlong_dtype dtype, void* stream);
 
+/* Variable-length batch: B independent sequences of lengths lens[b] (host
+ * array, 1 <= lens[b] <= Lmax), each with its own G = G(lens[b]) (Metodologia
+ * 1: G follows each sequence's current length), in padded tensors
+ *   q, out [B,Hq,Lmax,d], k, v [B,Hkv,Lmax,d]: rows [0, lens[b]) of sequence b
+ *   are used; out rows >= lens[b] are not written.  Padding rows of v must
+ *   hold finite values (they meet P = 0 in the P.V product).
+ *   lse (optional, may be NULL): float [B,Hq,Lmax] device array, 4-byte
+ *   aligned; row i of sequence b receives log sum_j exp(scale * logit_ij)
+ *   (natural log; the statistic an LSE merge of partial attentions needs).
+ * Other arguments and errors as jetlong_prefill; one launch per sequence. */
+int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int Hq, int Hkv, const int32_t* lens, int Lmax, int d,
+                           int w0, int w_pretrained, double rope_theta, float scale,
+                           jetlong_dtype dtype, void* stream);
+
 /* Bytes of device workspace jetlong_decode needs for any L <= Lcap with these
  * sizes (partial softmax states of the key splits plus merge counters).
  * Returns 0 for invalid sizes. */

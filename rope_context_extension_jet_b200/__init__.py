@@ -62,6 +62,9 @@ def load_library(path: str | None = None):
         lib.jetlong_prefill.restype = i32
         lib.jetlong_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                         dbl, flt, i32, vp]
+        lib.jetlong_prefill_varlen.restype = i32
+        lib.jetlong_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, i32, i32,
+                                               i32, dbl, flt, i32, vp]
         lib.jetlong_prefill_chunk.restype = i32
         lib.jetlong_prefill_chunk.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                               i32, i32, dbl, flt, i32, vp]
@@ -180,6 +183,36 @@ def prefill_chunk(q, kcache, vcache, P: int, out=None, *, w0: int, w_pretrained:
                                      int(w_pretrained), float(rope_theta), float(scale),
                                      _dtype_code(q), _stream(stream)), lib)
     return out
+
+
+def prefill_varlen(q, k, v, lens, out=None, *, w0: int, w_pretrained: int, rope_theta: float,
+                   scale: float | None = None, with_lse: bool = False, stream=None):
+    """Variable-length batch in padded tensors q/out [B,Hq,Lmax,d], k/v
+    [B,Hkv,Lmax,d]; sequence b uses rows [0, lens[b]) and its own G.  With
+    ``with_lse`` also returns the per-row natural-log LSE [B,Hq,Lmax] (fp32;
+    rows past a sequence's length are left as allocated)."""
+    import numpy as _np
+    import torch
+    B, Hq, Lmax, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, Lmax, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, Lmax, d] matching q")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    lens = _np.ascontiguousarray(_np.asarray(lens, dtype=_np.int32).reshape(-1))
+    if lens.shape[0] != B:
+        raise ValueError("lens must have one length per sequence")
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lmax), dtype=torch.float32, device=q.device) if with_lse else None
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_prefill_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
+                                      lse.data_ptr() if lse is not None else None, B, Hq, Hkv,
+                                      lens.ctypes.data, Lmax, d, int(w0), int(w_pretrained),
+                                      float(rope_theta), float(scale), _dtype_code(q),
+                                      _stream(stream)), lib)
+    return (out, lse) if with_lse else out
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, Lcap: int, d: int) -> int:

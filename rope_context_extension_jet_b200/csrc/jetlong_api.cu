@@ -127,9 +127,10 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
     return ok();
 }
 
-static int prefill_entry(const void* q, const void* k, const void* v, void* out, int B, int Hq,
-                         int Hkv, int P, int C, int Lcap, int d, int w0, int w_pretrained,
-                         double rope_theta, float scale, jetlong_dtype dtype, void* stream)
+static int prefill_entry(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                         int Hq, int Hkv, int P, int C, int Cst, int Lcap, int d, int w0,
+                         int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
+                         void* stream)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -147,7 +148,8 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     jl::PrefillProblem p{};
     p.q = q; p.k = k; p.v = v; p.out = out;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.d = d;
-    p.P = P; p.C = C; p.Lcap = Lcap;
+    p.P = P; p.C = C; p.Cst = Cst; p.Lcap = Lcap;
+    p.lse = lse;
     p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
     p.G = (int)jetlong_group_size(L, w_pretrained);
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -167,16 +169,41 @@ int jetlong_prefill(const void* q, const void* k, const void* v, void* out, int 
                     float scale, jetlong_dtype dtype, void* stream)
 {
     if (L < 1) return fail(JETLONG_ERR_INVALID_ARG, "L must be >= 1 (got %d)", L);
-    return prefill_entry(q, k, v, out, B, Hq, Hkv, 0, L, L, d, w0, w_pretrained, rope_theta, scale,
-                         dtype, stream);
+    return prefill_entry(q, k, v, out, nullptr, B, Hq, Hkv, 0, L, L, L, d, w0, w_pretrained,
+                         rope_theta, scale, dtype, stream);
 }
 
 int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache, void* out, int B,
                           int Hq, int Hkv, int P, int C, int Lcap, int d, int w0, int w_pretrained,
                           double rope_theta, float scale, jetlong_dtype dtype, void* stream)
 {
-    return prefill_entry(q, kcache, vcache, out, B, Hq, Hkv, P, C, Lcap, d, w0, w_pretrained,
-                         rope_theta, scale, dtype, stream);
+    return prefill_entry(q, kcache, vcache, out, nullptr, B, Hq, Hkv, P, C, C, Lcap, d, w0,
+                         w_pretrained, rope_theta, scale, dtype, stream);
+}
+
+int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                           int Hq, int Hkv, const int32_t* lens, int Lmax, int d, int w0,
+                           int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
+                           void* stream)
+{
+    if (!lens) return fail(JETLONG_ERR_INVALID_ARG, "null lens");
+    if (B < 1 || Lmax < 1) return fail(JETLONG_ERR_INVALID_ARG, "need B >= 1 and Lmax >= 1");
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 1 || lens[b] > Lmax)
+            return fail(JETLONG_ERR_INVALID_ARG, "lens[%d] = %d outside [1, Lmax = %d]", b, lens[b], Lmax);
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(JETLONG_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    const size_t el = dtype == JETLONG_FP32 ? 4 : 2;
+    for (int b = 0; b < B; ++b) {
+        // sequence b: its own planes, its own length and G, one launch
+        const size_t qo = (size_t)b * Hq * Lmax * d * el, ko = (size_t)b * Hkv * Lmax * d * el;
+        int st = prefill_entry(static_cast<const char*>(q) + qo, static_cast<const char*>(k) + ko,
+                               static_cast<const char*>(v) + ko, static_cast<char*>(out) + qo,
+                               lse ? lse + (size_t)b * Hq * Lmax : nullptr, 1, Hq, Hkv, 0, lens[b], Lmax,
+                               Lmax, d, w0, w_pretrained, rope_theta, scale, dtype, stream);
+        if (st != JETLONG_OK) return st;
+    }
+    return ok();
 }
 
 size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int Lcap, int d)

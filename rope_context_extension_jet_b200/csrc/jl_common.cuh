@@ -87,13 +87,16 @@ template <> __device__ __forceinline__ void store_elem<__nv_bfloat16>(__nv_bfloa
 // Host-side launch plumbing shared by the translation units.
 
 // Prefill of query rows at positions [P, P + C) against keys [0, L), L = P + C
-// (a whole sequence: P = 0, C = L).  q and out hold C rows per (b, head); k and
-// v hold Lcap >= L rows per (b, kv head), rows [0, L) valid.
+// (a whole sequence: P = 0, C = L).  q and out hold Cst >= C rows per (b, head)
+// (rows [0, C) used); k and v hold Lcap >= L rows per (b, kv head), rows [0, L)
+// valid.  lse (optional, may be null): Cst floats per (b, head), row r receives
+// the natural log of row r's softmax denominator.
 struct PrefillProblem {
     const void *q, *k, *v;
     void* out;
+    float* lse;
     int B, Hq, Hkv, L, d, w0;
-    int P, C, Lcap;
+    int P, C, Cst, Lcap;
     int G;             // dynamic group size for this call (fits int: G <= L)
     float scale_log2;  // scale * log2(e): logits kept in base-2 units
     RopeTurns turns;

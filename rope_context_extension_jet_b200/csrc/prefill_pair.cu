@@ -316,7 +316,7 @@ cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
 {
     CUtensorMap tq, tk, tv;
     cudaError_t e;
-    if ((e = make_map(&tq, pp.q, D, pp.C, pp.C, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tq, pp.q, D, pp.C, pp.Cst, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
     if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, KROWS)) != cudaSuccess) return e;
     if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);

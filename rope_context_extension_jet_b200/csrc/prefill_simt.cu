@@ -50,10 +50,11 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
     const int G = p.G;
 
     // query row i (position P + r of the chunk) is row i - P of q and out
-    const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * (size_t)p.C * D;
+    const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * (size_t)p.Cst * D;
     const T* k = reinterpret_cast<const T*>(p.k) + ((size_t)b * p.Hkv + kvh) * (size_t)p.Lcap * D;
     const T* v = reinterpret_cast<const T*>(p.v) + ((size_t)b * p.Hkv + kvh) * (size_t)p.Lcap * D;
-    T* out = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + h) * (size_t)p.C * D;
+    T* out = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + h) * (size_t)p.Cst * D;
+    float* lse = p.lse ? p.lse + ((size_t)b * p.Hq + h) * (size_t)p.Cst : nullptr;
 
     // Q tile, rotated at i and at floor(i/G), pre-scaled into base-2 logit units.
     for (int e = tid; e < BM * H; e += NT) {
@@ -236,6 +237,8 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
         float inv = 1.f / lrow[a];
 #pragma unroll
         for (int c = 0; c < CPT; ++c) store_elem(out + (size_t)(i - p.P) * D + tx + 16 * c, o[a][c] * inv);
+        // natural log of the softmax denominator (mrow, lrow are base-2 quantities)
+        if (lse && tx == 0) lse[i - p.P] = (mrow[a] + __log2f(lrow[a])) * 0.69314718055994531f;
     }
 }
 

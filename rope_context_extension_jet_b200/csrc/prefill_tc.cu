@@ -299,7 +299,7 @@ cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
 {
     CUtensorMap tq, tk, tv;
     cudaError_t e;
-    if ((e = make_map(&tq, pp.q, D, pp.C, pp.C, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
+    if ((e = make_map(&tq, pp.q, D, pp.C, pp.Cst, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
     if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);
@@ -364,12 +364,13 @@ TcParams make_params(const PrefillProblem& pp)
 {
     TcParams p{};
     p.B = pp.B; p.Hq = pp.Hq; p.Hkv = pp.Hkv; p.L = pp.L; p.w0 = pp.w0; p.G = pp.G;
-    p.P = pp.P; p.C = pp.C;
+    p.P = pp.P; p.C = pp.C; p.Cst = pp.Cst;
     p.nqb = (pp.C + BM - 1) / BM;
     make_div_magic((uint32_t)pp.G, &p.div_m, &p.div_s1, &p.div_s2);
     p.scale_log2 = pp.scale_log2;
     p.turns = pp.turns;
     p.out = reinterpret_cast<__nv_bfloat16*>(pp.out);
+    p.lse = pp.lse;
     p.dev_error = pp.dev_error;
     return p;
 }

@@ -32,11 +32,12 @@ enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
 // keys [0, L), L = P + C; nqb query blocks of BM rows.
 struct TcParams {
     int B, Hq, Hkv, L, w0, G, nqb;
-    int P, C;
+    int P, C, Cst;  // Cst: q / out / lse rows per (b, head) in memory
     uint32_t div_m, div_s1, div_s2;  // floor(x / G) by multiply-shift
     float scale_log2;
     RopeTurns turns;
     __nv_bfloat16* out;
+    float* lse;  // optional
     int* dev_error;
 };
 
@@ -317,7 +318,10 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
     if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, 0x333)) {
         tc_fence_after();
         const float inv = 1.f / l;
-        __nv_bfloat16* orow = p.out + (((size_t)b * p.Hq + head) * (size_t)p.C + (size_t)(i - p.P)) * D;
+        const size_t row = ((size_t)b * p.Hq + head) * (size_t)p.Cst + (size_t)(i - p.P);
+        __nv_bfloat16* orow = p.out + row * D;
+        // natural log of the softmax denominator: (m + log2 l) * ln 2 (m, l in base 2)
+        if (p.lse && i < L) p.lse[row] = (m_used + __log2f(l)) * 0.69314718055994531f;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t tt[32];

@@ -149,3 +149,23 @@ def test_decode_rope_cache_rejects_bad_arguments_on_host(lib, kw, status):
                                        a["scale"], a["dtype"], a["ws"], a["wsb"], NULL)
     assert st == status
     assert jl.launch_count() == before
+
+
+@pytest.mark.parametrize("lens,kw,status", [
+    ([10, 20], dict(), None), ([0, 20], dict(), 1), ([10, 65], dict(), 1), (None, dict(), 1),
+    ([10, 20], dict(q=NULL), 1), ([10, 20], dict(lse=ctypes.c_void_p((1 << 20) + 2)), 1),
+    ([10, 20], dict(d=96), 2),
+])
+def test_prefill_varlen_rejects_bad_arguments_on_host(lib, lens, kw, status):
+    a = dict(q=P, k=P, v=P, out=P, lse=NULL, B=2, Hq=4, Hkv=2, Lmax=64, d=128, w0=8, wp=32,
+             theta=1e6, scale=0.088, dtype=0)
+    a.update(kw)
+    arr = (ctypes.c_int32 * 2)(*lens) if lens is not None else None
+    if status is None:
+        return  # valid arguments would launch; covered by the GPU tests
+    before = jl.launch_count()
+    st = lib.jetlong_prefill_varlen(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"],
+                                    a["Hkv"], arr, a["Lmax"], a["d"], a["w0"], a["wp"], a["theta"],
+                                    a["scale"], a["dtype"], NULL)
+    assert st == status
+    assert jl.launch_count() == before

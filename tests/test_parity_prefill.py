@@ -246,3 +246,50 @@ def test_chunk_of_128k_sequence_sampled():
             list(range(0, 8)) + list(range(C - 8, C)) + list(rng.integers(0, C, 8))]
     chunk_case("chunk-128k", P, C, P + C, B=1, Hq=32, Hkv=8, d=128, w_pre=32768, w0=4096, index=69,
                rows=rows)
+
+
+# ---------------------------------------------------------------- variable-length batch + LSE
+# jetlong_prefill_varlen: sequence b of a padded batch uses rows [0, lens[b]) and
+# its own G; reference: the oracle's prefill of that sequence alone.  The LSE
+# (natural log of each row's softmax denominator) is a scaled-logit quantity, so
+# it takes the output gates' max-abs bound: 2e-2 for bf16 (fp16 logit operands),
+# 1e-4 for fp32.
+
+def varlen_case(name, lens, *, dtype="bf16", Hq=4, Hkv=1, d=128, w_pre=100, w0=17, theta=1e6,
+                index=70, pad=5):
+    import torch
+    B, Lmax = len(lens), max(lens) + pad
+    w = I.PrefillWorkload(name, index, dtype, B, Hq, Hkv, d, Lmax, w_pre, w0, theta)
+    q, k, v = I.prefill_inputs(w)
+    qd = to_device(q)
+    out = torch.full_like(qd, float("nan"))
+    out, lse = jl.prefill_varlen(qd, to_device(k), to_device(v), lens, out, w0=w0, w_pretrained=w_pre,
+                                 rope_theta=theta, scale=w.scale, with_lse=True)
+    jl.device_status()
+    got, got_lse = to_host_f64(out), lse.double().cpu().numpy()
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    for b, Lb in enumerate(lens):
+        hh, ii = np.meshgrid(np.arange(Hq), np.arange(Lb), indexing="ij")
+        rows = np.stack([np.zeros(hh.size, np.int32), hh.ravel(), ii.ravel()], axis=1)
+        sl = lambda a: np.ascontiguousarray(a[b:b + 1, :, :Lb])
+        ref, ref_lse = oracle.prefill_rows(sl(q), sl(k), sl(v), rows, w0=w0, w_pretrained=w_pre,
+                                           rope_theta=theta, scale=w.scale, with_lse=True)
+        check_gate(got[b, :, :Lb].reshape(-1, d), ref, dtype, f"{name} seq {b}")
+        assert np.abs(got_lse[b, :, :Lb].reshape(-1) - ref_lse).max() <= tol, f"{name} lse seq {b}"
+        assert np.isnan(got[b, :, Lb:]).all(), "rows past a sequence's length must stay untouched"
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 1), (4, 2), (3, 3)])
+def test_varlen_bf16(Hq, Hkv):
+    varlen_case(f"varlen-{Hq}-{Hkv}", [1000, 37, 513, 1, 130], Hq=Hq, Hkv=Hkv, w_pre=120, w0=64, index=71)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_fp32(d):
+    varlen_case(f"varlen-f32-{d}", [300, 1, 129], dtype="fp32", Hq=2, Hkv=1, d=d, w_pre=50, w0=20,
+                index=72)
+
+
+def test_varlen_lengths_cross_group_sizes():
+    # w_pretrained = 256: G = 1, 2, 4, 5 for the four sequences
+    varlen_case("varlen-G", [256, 257, 1024, 1025], Hq=8, Hkv=2, w_pre=256, w0=100, index=73)
