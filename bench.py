@@ -421,6 +421,28 @@ def main():
     plain_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in pl_ev])))
     _, plain_computed, _, _ = prefill_flops(wplain)
 
+    # ---------------- the pages' three-pass inclusion-exclusion form of the same
+    # prefill (jetlong_prefill_ie), outside the timed region: one pass against three
+    ie_ws = torch.empty(int(jl.load_library().jetlong_prefill_ie_workspace_size(wp.B, wp.Hq, wp.L, wp.d, 0)),
+                        dtype=torch.uint8, device=dev)
+
+    def ie_call():
+        jl.prefill_ie(qd, kd, vd, outd, w0=wp.w0, w_pretrained=wp.w_pretrained, rope_theta=wp.rope_theta,
+                      scale=wp.scale, workspace=ie_ws, stream=stream)
+
+    ie_call()
+    ie_ev = []
+    for _ in range(2):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ie_call()
+        b.record(stream)
+        ie_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    jl.device_status(stream)
+    ie_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ie_ev])))
+    del ie_ws
+
     # ---------------- chunked prefill (jetlong_prefill_chunk): the last 8192 rows
     # of the same 128K sequence as one chunk over the resident K/V, outside the
     # timed region
@@ -508,6 +530,8 @@ def main():
                         "chunk_last_8192_rows": {
                             "P": P_ch, "C": wp.L - P_ch, "ms": round(ch_ms, 3),
                             "tflops_computed": round(whole_job_rate(ch_computed, world, ch_ms * 1e-3) / 1e12, 2)},
+                        "inclusion_exclusion_three_pass": {
+                            "ms": round(ie_ms, 3), "three_pass_over_one_pass_time": round(ie_ms / pre_ms, 4)},
                         "plain_rope_same_kernel": {
                             "w0": wplain.w0, "ms": round(plain_ms, 3),
                             "tflops_computed": round(whole_job_rate(plain_computed, world, plain_ms * 1e-3) / 1e12, 2),

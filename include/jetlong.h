@@ -110,6 +110,22 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
                            int w0, int w_pretrained, double rope_theta, float scale,
                            jetlong_dtype dtype, void* stream);
 
+/* The pages' own formulation of the prefill (Metodologia 2, inclusion-
+ * exclusion): three standard attention passes -- A: window pairs (i - j < w0)
+ * at the exact positions, B: all causal pairs at the aliased positions, C:
+ * window pairs at the aliased positions -- merged per row with their softmax
+ * denominators, out = (e^lA O_A + e^lB O_B - e^lC O_C) / (e^lA + e^lB - e^lC).
+ * The result equals jetlong_prefill's up to rounding; it exists to compare
+ * the two forms.  Arguments as jetlong_prefill, plus a device workspace of at
+ * least jetlong_prefill_ie_workspace_size(B, Hq, L, d, dtype) bytes (16-byte
+ * aligned, caller-owned; the three pass outputs and their LSEs).  Four
+ * launches (one when w0 = 0: pass B alone). */
+size_t jetlong_prefill_ie_workspace_size(int B, int Hq, int L, int d, jetlong_dtype dtype);
+int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
+                       int B, int Hq, int Hkv, int L, int d,
+                       int w0, int w_pretrained, double rope_theta, float scale,
+                       jetlong_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace jetlong_decode needs for any L <= Lcap with these
  * sizes (partial softmax states of the key splits plus merge counters).
  * Returns 0 for invalid sizes. */

@@ -62,6 +62,11 @@ def load_library(path: str | None = None):
         lib.jetlong_prefill.restype = i32
         lib.jetlong_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                         dbl, flt, i32, vp]
+        lib.jetlong_prefill_ie_workspace_size.restype = sz
+        lib.jetlong_prefill_ie_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        lib.jetlong_prefill_ie.restype = i32
+        lib.jetlong_prefill_ie.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, dbl, flt,
+                                           i32, vp, sz, vp]
         lib.jetlong_prefill_varlen.restype = i32
         lib.jetlong_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, i32, i32,
                                                i32, dbl, flt, i32, vp]
@@ -182,6 +187,29 @@ def prefill_chunk(q, kcache, vcache, P: int, out=None, *, w0: int, w_pretrained:
                                      _dev(out, "out"), B, Hq, Hkv, int(P), C, Lcap, d, int(w0),
                                      int(w_pretrained), float(rope_theta), float(scale),
                                      _dtype_code(q), _stream(stream)), lib)
+    return out
+
+
+def prefill_ie(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: float,
+               scale: float | None = None, workspace=None, stream=None):
+    """The pages' three-pass inclusion-exclusion form of the prefill (same
+    result as ``prefill``; for comparing the two forms)."""
+    import torch
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, L, d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    lib = load_library()
+    need = int(lib.jetlong_prefill_ie_workspace_size(B, Hq, L, d, _dtype_code(q)))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    _check(lib.jetlong_prefill_ie(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), B, Hq,
+                                  Hkv, L, d, int(w0), int(w_pretrained), float(rope_theta),
+                                  float(scale), _dtype_code(q), _dev(workspace, "workspace"),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)), lib)
     return out
 
 

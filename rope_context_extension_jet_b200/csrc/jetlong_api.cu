@@ -130,7 +130,7 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
 static int prefill_entry(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                          int Hq, int Hkv, int P, int C, int Cst, int Lcap, int d, int w0,
                          int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
-                         void* stream)
+                         void* stream, int window_rot = -1)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -150,6 +150,7 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.d = d;
     p.P = P; p.C = C; p.Cst = Cst; p.Lcap = Lcap;
     p.lse = lse;
+    p.window_rot = window_rot;
     p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
     p.G = (int)jetlong_group_size(L, w_pretrained);
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -203,6 +204,70 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
                                Lmax, d, w0, w_pretrained, rope_theta, scale, dtype, stream);
         if (st != JETLONG_OK) return st;
     }
+    return ok();
+}
+
+// Workspace of the three-pass form: O_A, O_B, O_C in the output dtype, then
+// their per-row LSEs (fp32), each segment 256-byte aligned.
+static size_t ie_segments(int B, int Hq, int L, int d, jetlong_dtype dtype, size_t* o_bytes, size_t* l_bytes)
+{
+    const size_t el = dtype == JETLONG_FP32 ? 4 : 2;
+    *o_bytes = (((size_t)B * Hq * L * d * el) + 255) & ~(size_t)255;
+    *l_bytes = (((size_t)B * Hq * L * 4) + 255) & ~(size_t)255;
+    return 3 * (*o_bytes + *l_bytes);
+}
+
+size_t jetlong_prefill_ie_workspace_size(int B, int Hq, int L, int d, jetlong_dtype dtype)
+{
+    if (B < 1 || Hq < 1 || L < 1 || (d != 64 && d != 128)) return 0;
+    if (dtype != JETLONG_BF16 && dtype != JETLONG_FP32) return 0;
+    size_t ob, lb;
+    return ie_segments(B, Hq, L, d, dtype, &ob, &lb);
+}
+
+int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                       int L, int d, int w0, int w_pretrained, double rope_theta, float scale,
+                       jetlong_dtype dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!workspace) return fail(JETLONG_ERR_INVALID_ARG, "null workspace");
+    if (!aligned16(workspace)) return fail(JETLONG_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    if (L < 1) return fail(JETLONG_ERR_INVALID_ARG, "L must be >= 1 (got %d)", L);
+    int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
+    if (st != JETLONG_OK) return st;
+    size_t ob, lb;
+    const size_t need = ie_segments(B, Hq, L, d, dtype, &ob, &lb);
+    if (workspace_bytes < need)
+        return fail(JETLONG_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)", workspace_bytes, need);
+    char* ws = static_cast<char*>(workspace);
+    void* oa = ws;
+    void* obuf = ws + ob;
+    void* oc = ws + 2 * ob;
+    float* la = reinterpret_cast<float*>(ws + 3 * ob);
+    float* lbuf = reinterpret_cast<float*>(ws + 3 * ob + lb);
+    float* lc = reinterpret_cast<float*>(ws + 3 * ob + 2 * lb);
+    // B: every causal pair at the aliased positions (the routed kernel with w0 = 0)
+    st = prefill_entry(q, k, v, obuf, lbuf, B, Hq, Hkv, 0, L, L, L, d, 0, w_pretrained, rope_theta, scale,
+                       dtype, stream);
+    if (st != JETLONG_OK) return st;
+    if (w0 == 0) {
+        // no window: the routed output is pass B alone (A and C hold no pairs)
+        cudaError_t e = cudaMemcpyAsync(out, obuf, (size_t)B * Hq * L * d * (dtype == JETLONG_FP32 ? 4 : 2),
+                                        cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+        if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "copy: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    // A: window pairs at the exact positions; C: window pairs at the aliased positions
+    st = prefill_entry(q, k, v, oa, la, B, Hq, Hkv, 0, L, L, L, d, w0, w_pretrained, rope_theta, scale, dtype,
+                       stream, 0);
+    if (st != JETLONG_OK) return st;
+    st = prefill_entry(q, k, v, oc, lc, B, Hq, Hkv, 0, L, L, L, d, w0, w_pretrained, rope_theta, scale, dtype,
+                       stream, 1);
+    if (st != JETLONG_OK) return st;
+    int n = 0;
+    cudaError_t e = jl::launch_ie_merge(oa, obuf, oc, la, lbuf, lc, out, (long long)B * Hq * L, d, dtype,
+                                        (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

@@ -97,6 +97,10 @@ struct PrefillProblem {
     float* lse;
     int B, Hq, Hkv, L, d, w0;
     int P, C, Cst, Lcap;
+    // -1: the routed (bifocal) attention.  0 / 1: a plain windowed attention
+    // over the pairs with i - j < w0 only, every pair rotated to its exact (0)
+    // or aliased (1) positions (passes of the pages' inclusion-exclusion form).
+    int window_rot;
     int G;             // dynamic group size for this call (fits int: G <= L)
     float scale_log2;  // scale * log2(e): logits kept in base-2 units
     RopeTurns turns;
@@ -127,6 +131,11 @@ cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cuda
                                   int* nlaunch, size_t* need_bytes);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d);
 cudaError_t launch_position_map(int32_t* out, int L, int G, cudaStream_t s, int* nlaunch);
+// Inclusion-exclusion merge of three attention passes (A, B, C) with their
+// per-row LSEs: out = (e^lA O_A + e^lB O_B - e^lC O_C) / (e^lA + e^lB - e^lC).
+cudaError_t launch_ie_merge(const void* oa, const void* ob, const void* oc, const float* la, const float* lb,
+                            const float* lc, void* out, long long rows, int d, jetlong_dtype dt,
+                            cudaStream_t s, int* nlaunch);
 cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStream_t s, int* nlaunch);
 
 }  // namespace jl

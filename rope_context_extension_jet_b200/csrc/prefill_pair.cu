@@ -110,6 +110,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         mbar_init(&bars[P_DRAIN], 1);
         *abort_flag = 0;
         *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
+        if (p.window_rot >= 0) plan->nR = 0;  // windowed pass: the local tiles only
         // after a bounded wait expired anywhere in the grid (error word set),
         // later pairs skip their work; CTA 0 decides for both
         if (leader) *skip_word = *reinterpret_cast<volatile int*>(p.dev_error) != 0;
@@ -258,7 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, 0x431);
         if (ok) {
             for (int h = 0; h < 2; ++h) {
-                if (nR > 0)
+                if (nR > 0 || p.window_rot == 1)
                     rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
                 else
                     rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
@@ -283,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (!warp_wait(&bars[P_KFULL + s], u & 1, abort_flag, p.dev_error, 0x433)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
             unsigned char* kt = smem + S::K0 + s * S::KTILE;
-            if (e < nR)
+            if (e < nR || p.window_rot == 1)
                 rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
             else
                 rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts);

@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
     const int h = blockIdx.y, b = blockIdx.z;
     const int kvh = h / (p.Hq / p.Hkv);
     const int G = p.G;
+    const bool window = p.window_rot >= 0;  // windowed pass: local pairs only, one rotation
+    // positions of the "exact" rotation: i / j, or i / G, j / G in a windowed aliased pass
+    auto pe = [&](int x) { return (uint32_t)(p.window_rot == 1 ? x / G : x); };
 
     // query row i (position P + r of the chunk) is row i - P of q and out
     const T* q = reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * (size_t)p.Cst * D;
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
             bb = load_elem(q + (size_t)(i - p.P) * D + m + H);
         }
         float c, s;
-        rope_cs_accurate((uint32_t)i, p.turns.hi[m], p.turns.lo[m], c, s);
+        rope_cs_accurate(pe(i), p.turns.hi[m], p.turns.lo[m], c, s);
         sQe[r * QS + m] = (a * c - bb * s) * p.scale_log2;
         sQe[r * QS + m + H] = (a * s + bb * c) * p.scale_log2;
         rope_cs_accurate((uint32_t)(i / G), p.turns.hi[m], p.turns.lo[m], c, s);
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
         const int dmax = i_hi - j_lo;
         const int dmin = max(0, i_lo - j_hi);
         const bool need_loc = dmax >= 0 && dmin < p.w0;          // some pair is local
-        const bool need_rem = dmax >= p.w0;                      // some pair is remote
+        const bool need_rem = !window && dmax >= p.w0;           // some pair is remote
+        if (window && !need_loc) continue;  // uniform over the CTA: no local pair here
         __syncthreads();  // previous tile's K/V/P consumers are done
         for (int e = tid; e < BN * H; e += NT) {
             int r = e / H, m = e % H;
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
             }
             float c, s;
             if (need_loc) {
-                rope_cs_accurate((uint32_t)j, p.turns.hi[m], p.turns.lo[m], c, s);
+                rope_cs_accurate(pe(j), p.turns.hi[m], p.turns.lo[m], c, s);
                 sKe[r * QS + m] = a * c - bb * s;
                 sKe[r * QS + m + H] = a * s + bb * c;
             }
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(PrefillProblem p)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 int j = j_lo + tx + 16 * c;
-                if (j > i || j >= p.L) s[a][c] = -INFINITY;
+                if (j > i || j >= p.L || (window && i - j >= p.w0)) s[a][c] = -INFINITY;
                 mx = fmaxf(mx, s[a][c]);
             }
 #pragma unroll

@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
+        if (p.window_rot >= 0) plan->nR = 0;  // windowed pass: the local tiles only
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, 0x321);
         if (ok) {
             for (int h = 0; h < NH; ++h) {
-                if (nR > 0)
+                if (nR > 0 || p.window_rot == 1)
                     rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
                 else
                     rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, 0x323)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN);
-            if (e < nR)
+            if (e < nR || p.window_rot == 1)
                 rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
             else
                 rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts);
@@ -371,6 +372,7 @@ TcParams make_params(const PrefillProblem& pp)
     p.turns = pp.turns;
     p.out = reinterpret_cast<__nv_bfloat16*>(pp.out);
     p.lse = pp.lse;
+    p.window_rot = pp.window_rot;
     p.dev_error = pp.dev_error;
     return p;
 }

@@ -37,7 +37,8 @@ struct TcParams {
     float scale_log2;
     RopeTurns turns;
     __nv_bfloat16* out;
-    float* lse;  // optional
+    float* lse;      // optional
+    int window_rot;  // -1 routed; 0 / 1: pairs i - j < w0 only, exact / aliased rotation
     int* dev_error;
 };
 

@@ -169,3 +169,15 @@ def test_prefill_varlen_rejects_bad_arguments_on_host(lib, lens, kw, status):
                                     a["scale"], a["dtype"], NULL)
     assert st == status
     assert jl.launch_count() == before
+
+
+def test_prefill_ie_workspace_and_arguments(lib):
+    assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 128, 0) >= 3 * (4 * 600 * 128 * 2 + 4 * 600 * 4)
+    assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 96, 0) == 0
+    before = jl.launch_count()
+    args = [P, P, P, P, 1, 4, 2, 64, 128, 8, 32, 1e6, 0.088, 0]
+    assert lib.jetlong_prefill_ie(*args, NULL, 1 << 30, NULL) == 1          # null workspace
+    assert lib.jetlong_prefill_ie(*args, P, 16, NULL) == 1                  # too small
+    args[5] = 3
+    assert lib.jetlong_prefill_ie(*args, P, 1 << 30, NULL) == 1             # Hq % Hkv
+    assert jl.launch_count() == before

@@ -293,3 +293,47 @@ def test_varlen_fp32(d):
 def test_varlen_lengths_cross_group_sizes():
     # w_pretrained = 256: G = 1, 2, 4, 5 for the four sequences
     varlen_case("varlen-G", [256, 257, 1024, 1025], Hq=8, Hkv=2, w_pre=256, w0=100, index=73)
+
+
+# ---------------------------------------------------------------- inclusion-exclusion form
+# jetlong_prefill_ie: the pages' three passes merged with their LSEs; the
+# reference is the same oracle (the merge is exact), at the same gates.
+
+def ie_case(name, *, dtype="bf16", B=1, Hq=4, Hkv=1, d=128, L=600, w_pre=100, w0=17, theta=1e6, index=80):
+    w = I.PrefillWorkload(name, index, dtype, B, Hq, Hkv, d, L, w_pre, w0, theta)
+    q, k, v = I.prefill_inputs(w)
+    out = jl.prefill_ie(to_device(q), to_device(k), to_device(v), w0=w0, w_pretrained=w_pre,
+                        rope_theta=theta, scale=w.scale)
+    jl.device_status()
+    ref = oracle.prefill(q, k, v, w0=w0, w_pretrained=w_pre, rope_theta=theta, scale=w.scale)
+    return check_gate(to_host_f64(out), ref, dtype, name)
+
+
+@pytest.mark.parametrize("w0", [0, 1, 17, 128, 300, 5000])
+def test_ie_windows_head_quads(w0):
+    ie_case(f"ie-q-{w0}", w0=w0, index=81)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (3, 3)])
+def test_ie_other_groups(Hq, Hkv):
+    ie_case(f"ie-g-{Hq}-{Hkv}", Hq=Hq, Hkv=Hkv, L=513, w0=130, index=82)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_ie_fp32(d):
+    ie_case(f"ie-f32-{d}", dtype="fp32", Hq=2, Hkv=1, d=d, L=300, w0=40, w_pre=64, index=83)
+
+
+def test_ie_equals_one_pass_at_128k_sampled():
+    """The headline workload in the three-pass form: sampled rows against the oracle."""
+    w = I.C4
+    q, k, v = I.prefill_inputs(w)
+    out = jl.prefill_ie(to_device(q), to_device(k), to_device(v), w0=w.w0, w_pretrained=w.w_pretrained,
+                        rope_theta=w.rope_theta, scale=w.scale)
+    jl.device_status()
+    rows = I.sampled_rows(w, heads=[0, 11, 22, 31])
+    got = to_host_f64(out[rows[:, 0], rows[:, 1], rows[:, 2]])
+    del out
+    ref = oracle.prefill_rows(q, k, v, rows, w0=w.w0, w_pretrained=w.w_pretrained,
+                              rope_theta=w.rope_theta, scale=w.scale)
+    check_gate(got, ref, "bf16", "ie-128k")
