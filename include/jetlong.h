@@ -126,6 +126,23 @@ int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
                        int w0, int w_pretrained, double rope_theta, float scale,
                        jetlong_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Prefill from host buffers with the transfers overlapped: the sequence is
+ * processed as nchunks chunks of query rows (whole 128-row blocks), and while
+ * chunk c computes (jetlong_prefill_chunk semantics over the rows uploaded so
+ * far) the rows of chunk c + 1 travel host -> device and those of chunk c - 1
+ * device -> host, on two copy streams the library keeps per device.
+ *   q_host, k_host, v_host, out_host: host tensors [B,H,L,d] (page-locked
+ *   memory for the copies to overlap); q_dev, k_dev, v_dev, out_dev: device
+ *   tensors of the same shapes, owned by the caller, 16-byte aligned.
+ *   nchunks >= 1; other arguments as jetlong_prefill.
+ * Asynchronous: work queued on `stream` afterwards runs after out_host is
+ * complete.  Same result as copying in, jetlong_prefill, copying out. */
+int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                             void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                             int B, int Hq, int Hkv, int L, int d,
+                             int w0, int w_pretrained, double rope_theta, float scale,
+                             jetlong_dtype dtype, int nchunks, void* stream);
+
 /* Bytes of device workspace jetlong_decode needs for any L <= Lcap with these
  * sizes (partial softmax states of the key splits plus merge counters).
  * Returns 0 for invalid sizes. */

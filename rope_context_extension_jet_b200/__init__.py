@@ -67,6 +67,9 @@ def load_library(path: str | None = None):
         lib.jetlong_prefill_ie.restype = i32
         lib.jetlong_prefill_ie.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, dbl, flt,
                                            i32, vp, sz, vp]
+        lib.jetlong_prefill_streamed.restype = i32
+        lib.jetlong_prefill_streamed.argtypes = [vp] * 8 + [i32, i32, i32, i32, i32, i32, i32, dbl, flt,
+                                                            i32, i32, vp]
         lib.jetlong_prefill_varlen.restype = i32
         lib.jetlong_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, i32, i32,
                                                i32, dbl, flt, i32, vp]
@@ -211,6 +214,39 @@ def prefill_ie(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: flo
                                   float(scale), _dtype_code(q), _dev(workspace, "workspace"),
                                   workspace.numel() * workspace.element_size(), _stream(stream)), lib)
     return out
+
+
+def _host(t, name):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def prefill_streamed(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, *, w0: int,
+                     w_pretrained: int, rope_theta: float, scale: float | None = None, nchunks: int = 16,
+                     stream=None):
+    """Prefill from (page-locked) host tensors into ``out_host`` with the transfers
+    overlapped with the compute, chunk by chunk; ``*_dev`` are device tensors of
+    the same shapes used as staging.  Asynchronous on ``stream``."""
+    B, Hq, L, d = q_host.shape
+    Hkv = k_host.shape[1]
+    for t, n in ((q_dev, "q_dev"), (out_dev, "out_dev"), (out_host, "out_host")):
+        if t.shape != q_host.shape or t.dtype != q_host.dtype:
+            raise ValueError(f"{n} must match q_host's shape and dtype")
+    for t, n in ((k_dev, "k_dev"), (v_dev, "v_dev"), (v_host, "v_host")):
+        if t.shape != k_host.shape or t.dtype != k_host.dtype:
+            raise ValueError(f"{n} must match k_host's shape and dtype")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    lib = load_library()
+    _check(lib.jetlong_prefill_streamed(_host(q_host, "q_host"), _host(k_host, "k_host"),
+                                        _host(v_host, "v_host"), _host(out_host, "out_host"),
+                                        _dev(q_dev, "q_dev"), _dev(k_dev, "k_dev"), _dev(v_dev, "v_dev"),
+                                        _dev(out_dev, "out_dev"), B, Hq, Hkv, L, d, int(w0),
+                                        int(w_pretrained), float(rope_theta), float(scale),
+                                        _dtype_code(q_host), int(nchunks), _stream(stream)), lib)
+    return out_host
 
 
 def prefill_varlen(q, k, v, lens, out=None, *, w0: int, w_pretrained: int, rope_theta: float,

@@ -9,8 +9,11 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "jl_common.cuh"
 
@@ -130,7 +133,7 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
 static int prefill_entry(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                          int Hq, int Hkv, int P, int C, int Cst, int Lcap, int d, int w0,
                          int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
-                         void* stream, int window_rot = -1)
+                         void* stream, int window_rot = -1, int g_len = 0)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -152,7 +155,9 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     p.lse = lse;
     p.window_rot = window_rot;
     p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
-    p.G = (int)jetlong_group_size(L, w_pretrained);
+    // G from the current length (a chunk's P + C), or from g_len when the chunk
+    // is part of one whole-sequence prefill
+    p.G = (int)jetlong_group_size(g_len > 0 ? g_len : L, w_pretrained);
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.dev_error = derr;
@@ -268,6 +273,89 @@ int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out, i
                                         (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+// Two non-blocking copy streams per device (host->device, device->host), made
+// once and kept for the process.
+static cudaError_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h)
+{
+    static std::mutex mu;
+    static std::map<int, std::pair<cudaStream_t, cudaStream_t>> per_device;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = per_device.find(dev);
+    if (it == per_device.end()) {
+        cudaStream_t a = nullptr, b = nullptr;
+        if ((e = cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        it = per_device.emplace(dev, std::make_pair(a, b)).first;
+    }
+    *h2d = it->second.first;
+    *d2h = it->second.second;
+    return cudaSuccess;
+}
+
+int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                             void* q_dev, void* k_dev, void* v_dev, void* out_dev, int B, int Hq, int Hkv,
+                             int L, int d, int w0, int w_pretrained, double rope_theta, float scale,
+                             jetlong_dtype dtype, int nchunks, void* stream)
+{
+    if (!q_host || !k_host || !v_host || !out_host)
+        return fail(JETLONG_ERR_INVALID_ARG, "null host tensor pointer");
+    if (!q_dev || !k_dev || !v_dev || !out_dev) return fail(JETLONG_ERR_INVALID_ARG, "null device tensor pointer");
+    if (L < 1 || nchunks < 1) return fail(JETLONG_ERR_INVALID_ARG, "need L >= 1 and nchunks >= 1");
+    int st = check_common(B, Hq, Hkv, d, w0, w_pretrained, rope_theta, scale, dtype);
+    if (st != JETLONG_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream, h2d, d2h;
+    cudaError_t e = copy_streams(&h2d, &d2h);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "copy streams: %s", cudaGetErrorString(e));
+    const size_t row = (size_t)d * (dtype == JETLONG_FP32 ? 4 : 2), pitch = (size_t)L * row;
+    // chunks of whole 128-row query blocks (the last one ragged)
+    int C0 = (L + nchunks - 1) / nchunks;
+    C0 = (C0 + 127) / 128 * 128;
+    const int nch = (L + C0 - 1) / C0;
+    std::vector<cudaEvent_t> ev(2 * nch + 2, nullptr);
+    for (auto& x : ev)
+        if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) break;
+    auto release = [&] {
+        for (auto& x : ev)
+            if (x) cudaEventDestroy(x);  // destruction waits for pending work on the event
+    };
+    if (e != cudaSuccess) { release(); return fail(JETLONG_ERR_CUDA, "events: %s", cudaGetErrorString(e)); }
+    auto cp = [&](void* dst, const void* src, int P, int C, int planes, cudaMemcpyKind kind, cudaStream_t s2) {
+        return cudaMemcpy2DAsync(static_cast<char*>(dst) + (size_t)P * row, pitch,
+                                 static_cast<const char*>(src) + (size_t)P * row, pitch, (size_t)C * row,
+                                 (size_t)planes, kind, s2);
+    };
+    // the copies start after the work already queued on the caller's stream
+    if ((e = cudaEventRecord(ev[0], cs)) == cudaSuccess && (e = cudaStreamWaitEvent(h2d, ev[0], 0)) == cudaSuccess)
+        e = cudaStreamWaitEvent(d2h, ev[0], 0);
+    for (int c = 0; c < nch && e == cudaSuccess && st == JETLONG_OK; ++c) {
+        const int P = c * C0, C = L - P < C0 ? L - P : C0;
+        // rows [P, P + C) of every plane in; the chunk's prefill (keys [0, P + C),
+        // later rows of the device buffers are outside its tensor maps); rows out
+        if ((e = cp(q_dev, q_host, P, C, B * Hq, cudaMemcpyHostToDevice, h2d)) != cudaSuccess) break;
+        if ((e = cp(k_dev, k_host, P, C, B * Hkv, cudaMemcpyHostToDevice, h2d)) != cudaSuccess) break;
+        if ((e = cp(v_dev, v_host, P, C, B * Hkv, cudaMemcpyHostToDevice, h2d)) != cudaSuccess) break;
+        if ((e = cudaEventRecord(ev[1 + 2 * c], h2d)) != cudaSuccess) break;
+        if ((e = cudaStreamWaitEvent(cs, ev[1 + 2 * c], 0)) != cudaSuccess) break;
+        st = prefill_entry(static_cast<char*>(q_dev) + (size_t)P * row, k_dev, v_dev,
+                           static_cast<char*>(out_dev) + (size_t)P * row, nullptr, B, Hq, Hkv, P, C, L, L, d, w0,
+                           w_pretrained, rope_theta, scale, dtype, stream, -1, L);
+        if (st != JETLONG_OK) break;
+        if ((e = cudaEventRecord(ev[2 + 2 * c], cs)) != cudaSuccess) break;
+        if ((e = cudaStreamWaitEvent(d2h, ev[2 + 2 * c], 0)) != cudaSuccess) break;
+        e = cp(out_host, out_dev, P, C, B * Hq, cudaMemcpyDeviceToHost, d2h);
+    }
+    // the caller's stream continues once the last rows are back on the host
+    if (e == cudaSuccess && st == JETLONG_OK && (e = cudaEventRecord(ev[2 * nch + 1], d2h)) == cudaSuccess)
+        e = cudaStreamWaitEvent(cs, ev[2 * nch + 1], 0);
+    release();
+    if (st != JETLONG_OK) return st;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "streamed prefill: %s", cudaGetErrorString(e));
     return ok();
 }
 

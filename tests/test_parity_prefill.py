@@ -337,3 +337,28 @@ def test_ie_equals_one_pass_at_128k_sampled():
     ref = oracle.prefill_rows(q, k, v, rows, w0=w.w0, w_pretrained=w.w_pretrained,
                               rope_theta=w.rope_theta, scale=w.scale)
     check_gate(got, ref, "bf16", "ie-128k")
+
+
+# ---------------------------------------------------------------- host buffers, overlapped copies
+@pytest.mark.parametrize("L,nchunks,Hq,Hkv,dtype", [(1000, 3, 4, 1, "bf16"), (777, 16, 4, 2, "bf16"),
+                                                    (300, 2, 2, 1, "fp32"), (129, 8, 4, 1, "bf16")])
+def test_streamed_prefill_from_host(L, nchunks, Hq, Hkv, dtype):
+    import torch
+    w = I.PrefillWorkload(f"stream-{L}-{nchunks}", 90, dtype, 1, Hq, Hkv, 128, L, 200, 50, 1e6)
+    q, k, v = I.prefill_inputs(w)
+
+    def host(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.contiguous().pin_memory()
+
+    qh, kh, vh = host(q), host(k), host(v)
+    outh = torch.full_like(qh, float("nan")).pin_memory()
+    qd, kd, vd = (torch.empty_like(x, device="cuda") for x in (qh, kh, vh))
+    outd = torch.empty_like(qd)
+    jl.prefill_streamed(qh, kh, vh, outh, qd, kd, vd, outd, w0=w.w0, w_pretrained=w.w_pretrained,
+                        rope_theta=w.rope_theta, scale=w.scale, nchunks=nchunks)
+    torch.cuda.current_stream().synchronize()
+    jl.device_status()
+    ref = oracle.prefill(q, k, v, w0=w.w0, w_pretrained=w.w_pretrained, rope_theta=w.rope_theta,
+                         scale=w.scale)
+    check_gate(outh.double().numpy(), ref, dtype, w.name)
