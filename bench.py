@@ -422,6 +422,35 @@ def main():
     plain_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in pl_ev])))
     _, plain_computed, _, _ = prefill_flops(wplain)
 
+    # ---------------- the other configurations (PR1 fp32, C2 G = 1, C3 G = 2 with
+    # outlier keys): the same kernels on their shapes, outside the timed region
+    other = {}
+    for wo in (I.PR1, I.C2, I.C3):
+        qo, ko, vo = (to_dev(a, dev) for a in I.prefill_inputs(wo))
+        oo = torch.empty_like(qo)
+
+        def other_call():
+            jl.prefill(qo, ko, vo, oo, w0=wo.w0, w_pretrained=wo.w_pretrained, rope_theta=wo.rope_theta,
+                       scale=wo.scale, stream=stream)
+
+        other_call()
+        ev_o = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            other_call()
+            b.record(stream)
+            ev_o.append((a, b))
+        torch.cuda.synchronize(dev)
+        jl.device_status(stream)
+        ms_o = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev_o])))
+        u_o, c_o, _, _ = prefill_flops(wo)
+        other[wo.name] = {"ms": round(ms_o, 4), "dtype": wo.dtype,
+                          "tflops_computed": round(whole_job_rate(c_o, world, ms_o * 1e-3) / 1e12, 2),
+                          "tflops_useful": round(whole_job_rate(u_o, world, ms_o * 1e-3) / 1e12, 2),
+                          "tokens_per_s": round(world * wo.B * wo.L / (ms_o * 1e-3), 1)}
+        del qo, ko, vo, oo
+
     # ---------------- the pages' three-pass inclusion-exclusion form of the same
     # prefill (jetlong_prefill_ie), outside the timed region: one pass against three
     ie_ws = torch.empty(int(jl.load_library().jetlong_prefill_ie_workspace_size(wp.B, wp.Hq, wp.L, wp.d, 0)),
@@ -536,6 +565,7 @@ def main():
                             "w0": wplain.w0, "ms": round(plain_ms, 3),
                             "tflops_computed": round(whole_job_rate(plain_computed, world, plain_ms * 1e-3) / 1e12, 2),
                             "bifocal_over_plain_time": round(pre_ms / plain_ms, 4)}},
+            "other_prefill_configs": other,
             "decode": {"ms_per_token_step": round(dec_ms / wd.steps, 4),
                        "gbs_kv": round(dec_gbs, 1), "bytes_per_pass_kv": kv_bytes,
                        "bytes_per_pass_all": all_bytes, "tokens_per_s": round(dec_tok_s, 1),
