@@ -133,7 +133,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int nR = tp.nR, NE = tp.count();
 
     if (warp < 4) {
-        regs_dec<48>();
+        regs_dec<56>();
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
@@ -250,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
         }
     } else if (warp < 8) {
-        regs_dec<80>();
+        regs_dec<72>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
