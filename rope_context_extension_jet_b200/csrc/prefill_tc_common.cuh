@@ -203,7 +203,7 @@ __device__ __forceinline__ void rope_steps(int t, const TcParams& p, float (&stc
 // Softmax role of one query head: one thread per query row (= TMEM lane), 4
 // warps.  For each key tile e: wait for S = Q K^T in TMEM (`sfull`), apply the
 // causal / length / band masks, online softmax in base 2 with lazy O rescaling
-// (once the previous P.V finished, `pvdone`), write P (bf16) over the first 64
+// (after the previous P.V finished, `pvdone`), write P (bf16) over the first 64
 // columns of S and signal the MMA issuer (`arrive_p`); finally O / l -> out.
 // s_col / o_col are this warp's TMEM addresses of S and O.
 template <int D, bool CLUSTER, class ArriveP>
@@ -287,11 +287,14 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
             pk[(u >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
         }
         l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        if (e > 0) {
-            // previous P.V of this head finished: O is stable and P's columns are free
+        // The previous P.V of this head has finished: the MMA issuer issues it
+        // before Q K^T of this tile, whose commit (sfull) tracks every earlier
+        // MMA of that thread.  So P may overwrite its columns now; the rare O
+        // rescale still checks pvdone explicitly.
+        if (e > 0 && __any_sync(0xffffffffu, resc)) {
             if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, 0x332)) { ok = false; break; }
             tc_fence_after();
-            if (__any_sync(0xffffffffu, resc)) {
+            {
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t tt[32];
