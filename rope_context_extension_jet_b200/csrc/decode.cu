@@ -458,7 +458,7 @@ template <int D>
 __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int kw, int lane, uint32_t pa, uint32_t pb,
                                              float sgn, const uint2* sturns, const uint32_t (&qb)[D / 16][2])
 {
-    const int g = lane >> 2, t = lane & 3;
+    const int t = lane & 3;
     c[0] = c[1] = c[2] = c[3] = 0.f;
     // ldmatrix.x4 rows: lanes 0-7 keys 0-7 / chunk lo, 8-15 keys 8-15 / lo, 16-23 keys 0-7 / hi, 24-31 keys 8-15 / hi
     const int lkey = kw + (lane & 7) + ((lane >> 3) & 1) * 8, lhalf = lane >> 4;
@@ -659,7 +659,6 @@ __global__ void __launch_bounds__(TC_NT, 2)
             ldsm_x2_t(pbuf + (lane & 15) * 16, pb0, pb1);
             // O^T += V^T P^T over the d/16 row tiles of 16 dims
             const int vkey = kw + (lane & 7) + (lane >> 4) * 8, vhalf = (lane >> 3) & 1;
-#pragma unroll
             // keys past the valid range (cache rows >= L may hold anything) contribute
             // exactly zero: their V entries are cleared, not only their P
             const bool tail = jb + 15 >= j_end;

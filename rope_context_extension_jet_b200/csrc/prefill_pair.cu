@@ -22,7 +22,8 @@
 //
 // Roles (512 threads per CTA; registers rebalanced with setmaxnreg):
 //   warp 0      TMA producer (both CTAs): own Q tiles, own K and V halves
-//   warp 1      MMA issuer (CTA 0 only, one thread), cta_group::2
+//   warp 1      MMA issuer (CTA 0 only; the whole warp runs the loop, one
+//               elected lane issues each instruction), cta_group::2
 //   warp 2      TMEM allocation / release (cta_group::2, both CTAs)
 //   warp 3      CTA 1: tells CTA 0 when its V half landed
 //   warps 4-7   rotation of own Q tiles and own K halves
@@ -166,40 +167,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mbar_wait(&bars[P_QFULL], 0);
             for (int ee = max(0, k_issued - NS); ee < k_issued; ++ee) mbar_wait(&bars[P_KFULL + ee % NS], (ee / NS) & 1);
             for (int ee = max(0, v_issued - NS); ee < v_issued; ++ee) mbar_wait(&bars[P_VFULL + ee % NS], (ee / NS) & 1);
-        } else if (warp == 1 && lane == 0 && leader) {
+        } else if (warp == 1 && leader) {
             // ---------------------------------------------------------- MMA issuer
+            // Every value below is warp-uniform (the TMEM base is broadcast from
+            // lane 0), every wait is warp-collective, and each MMA / commit is
+            // issued by one elected lane.
             constexpr uint32_t IDESC_QK = idesc_f16(2 * BM, BN, 0);
             constexpr uint32_t IDESC_PV = idesc_bf16(2 * BM, D, 1);
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
             const uint32_t sbase = smem_u32(smem);
             auto qk = [&](int h, int s) {
                 const uint32_t qaddr = sbase + h * S::QTILE, kaddr = sbase + S::K0 + s * S::KTILE;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
-                    umma_pair_ss(tmem + h * 128, sdesc_sw128(qaddr + (k >> 2) * ATOM + (k & 3) * 32, 16, 1024),
-                                 sdesc_sw128(kaddr + (k >> 2) * S::KATOM + (k & 3) * 32, 16, 1024), IDESC_QK,
-                                 k > 0 ? 1u : 0u);
-                umma_commit_pair_both(&bars[P_SFULL + h]);
+                    umma_pair_ss_elect(tm + h * 128, sdesc_sw128(qaddr + (k >> 2) * ATOM + (k & 3) * 32, 16, 1024),
+                                       sdesc_sw128(kaddr + (k >> 2) * S::KATOM + (k & 3) * 32, 16, 1024), IDESC_QK,
+                                       k > 0 ? 1u : 0u);
+                umma_commit_pair_both_elect(&bars[P_SFULL + h]);
             };
             auto pv = [&](int h, int s, bool first) {
                 const uint32_t vaddr = sbase + S::V0 + s * S::VTILE;
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
-                    umma_pair_ts(tmem + 256 + h * 128, tmem + h * 128 + k * 8,
-                                 sdesc_sw128(vaddr + k * 2048, S::VTILE, 1024), IDESC_PV, (!first || k > 0) ? 1u : 0u);
-                umma_commit_pair_both(&bars[P_PVDONE + h]);
+                    umma_pair_ts_elect(tm + 256 + h * 128, tm + h * 128 + k * 8,
+                                       sdesc_sw128(vaddr + k * 2048, S::VTILE, 1024), IDESC_PV,
+                                       (!first || k > 0) ? 1u : 0u);
+                umma_commit_pair_both_elect(&bars[P_PVDONE + h]);
             };
             // V half of tile pe landed in both CTAs and P_h of tile pe is in both TMEMs
             auto pv_ready = [&](int h, int pe) {
                 const int s = pe % NS, u = pe / NS;
-                return wait_or_abort<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, 0x411 + h) &&
-                       (h == 1 || (wait_or_abort(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x413) &&
-                                   wait_or_abort<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, 0x414)));
+                return warp_wait<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, 0x411 + h) &&
+                       (h == 1 || (warp_wait(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x413) &&
+                                   warp_wait<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, 0x414)));
             };
             // Issue order per tile e: P_0 V (tile e-1), Q_0 K^T (tile e), P_1 V
             // (tile e-1), Q_1 K^T (tile e).  S_h(e) overwrites P_h(e-1) in TMEM;
-            // the P.V reading it was issued earlier by this thread and the
-            // tensor pipe runs one thread's MMAs in issue order.
-            bool ok = wait_or_abort<true>(&bars[P_QREADY0], 0, abort_flag, p.dev_error, 0x415);
+            // the P.V reading it was issued earlier by this warp and the tensor
+            // pipe runs one issuer's MMAs in issue order.
+            bool ok = warp_wait<true>(&bars[P_QREADY0], 0, abort_flag, p.dev_error, 0x415);
             tc_fence_after();
             for (int e = 0; e < NE && ok; ++e) {
                 const int s = e % NS, u = e / NS, pe = e - 1, ps = (e + NS - 1) % NS;
@@ -210,20 +216,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 }
                 if (e == nR && nR > 0) {
                     // Q of phase R is no longer read once every MMA so far completed
-                    umma_commit_pair_both(&bars[P_QFREE]);
-                    if (!wait_or_abort<true>(&bars[P_QREADY1], 0, abort_flag, p.dev_error, 0x416)) { ok = false; break; }
+                    umma_commit_pair_both_elect(&bars[P_QFREE]);
+                    if (!warp_wait<true>(&bars[P_QREADY1], 0, abort_flag, p.dev_error, 0x416)) { ok = false; break; }
                 }
-                if (!wait_or_abort<true>(&bars[P_KREADY + s], u & 1, abort_flag, p.dev_error, 0x417)) { ok = false; break; }
+                if (!warp_wait<true>(&bars[P_KREADY + s], u & 1, abort_flag, p.dev_error, 0x417)) { ok = false; break; }
                 tc_fence_after();
                 qk(0, s);
                 if (e > 0) {
                     if (!pv_ready(1, pe)) { ok = false; break; }
                     tc_fence_after();
                     pv(1, ps, pe == 0);
-                    umma_commit_pair_both(&bars[P_VEMPTY + ps]);
+                    umma_commit_pair_both_elect(&bars[P_VEMPTY + ps]);
                 }
                 qk(1, s);
-                umma_commit_pair_both(&bars[P_KEMPTY + s]);
+                umma_commit_pair_both_elect(&bars[P_KEMPTY + s]);
             }
             if (ok && NE > 0) {
                 const int pe = NE - 1, ps = pe % NS;
@@ -233,13 +239,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     if (pv_ready(1, pe)) {
                         tc_fence_after();
                         pv(1, ps, pe == 0);
-                        umma_commit_pair_both(&bars[P_VEMPTY + ps]);
+                        umma_commit_pair_both_elect(&bars[P_VEMPTY + ps]);
                     }
                 }
             }
-            // drain: every MMA issued by this thread completed before the pair
+            // drain: every MMA issued by this warp completed before the pair
             // meets at the closing cluster barrier
-            umma_commit_pair_local(&bars[P_DRAIN]);
+            umma_commit_pair_local_elect(&bars[P_DRAIN]);
             mbar_wait(&bars[P_DRAIN], 0);
         } else if (warp == 3 && lane == 0 && !leader) {
             // ---------------------------------------------------------- V relay (CTA 1)

@@ -217,6 +217,52 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar)
                  : "memory");
 }
 
+// Warp-collective forms of the pair MMA and commits: the whole (converged)
+// warp executes them with warp-uniform operands and one lane, chosen by
+// elect.sync, issues the instruction.  Keeping the issuing loop on a full warp
+// lets the descriptors live in uniform registers; a single divergent thread
+// pays a per-instruction detour to make its operands uniform.
+__device__ __forceinline__ void umma_pair_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_pair_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_both_elect(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+            smem_u32(bar)),
+        "h"((unsigned short)0x3)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local_elect(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 //   bits [0,14) start address >> 4; [16,30) leading byte offset >> 4;
 //   [32,46) stride byte offset >> 4; [46,48) version = 1; [49,52) base offset = 0;
