@@ -21,8 +21,9 @@ import threading
 
 __all__ = [
     "BF16", "FP32", "JetLongError", "load_library", "group_size", "position_map", "prefill",
-    "decode_workspace_size", "decode", "decode_noalloc", "device_status", "last_error",
-    "launch_count", "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout",
+    "prefill_chunk", "prefill_varlen", "prefill_ie", "prefill_streamed", "decode_workspace_size",
+    "decode", "decode_rope_cache", "decode_noalloc", "device_status", "last_error", "launch_count",
+    "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -120,11 +121,27 @@ def _dtype_code(t) -> int:
 
 
 def _dev(t, name):
+    import torch
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device} but the library runs on the current device "
+                         f"cuda:{torch.cuda.current_device()} (select it with torch.cuda.device)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _like(t, ref, name, ref_name):
+    """The library writes ``t`` with ``ref``'s shape and element type."""
+    if tuple(t.shape) != tuple(ref.shape) or t.dtype != ref.dtype:
+        raise ValueError(f"{name} must match {ref_name}: shape {tuple(ref.shape)}, dtype {ref.dtype} "
+                         f"(got {tuple(t.shape)}, {t.dtype})")
+
+
+def _same_dtype(*named):
+    if len({t.dtype for t, _ in named}) != 1:
+        raise TypeError(", ".join(n for _, n in named) + " must share a dtype")
 
 
 def last_error() -> str:
@@ -159,10 +176,10 @@ def prefill(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: float,
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
         raise ValueError("k and v must be [B, Hkv, L, d] matching q")
-    if not (q.dtype == k.dtype == v.dtype):
-        raise TypeError("q, k, v must share a dtype")
+    _same_dtype((q, "q"), (k, "k"), (v, "v"))
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
     _check(lib.jetlong_prefill(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"),
@@ -180,10 +197,10 @@ def prefill_chunk(q, kcache, vcache, P: int, out=None, *, w0: int, w_pretrained:
     _, Hkv, Lcap, _ = kcache.shape
     if vcache.shape != kcache.shape or kcache.shape[0] != B or kcache.shape[3] != d:
         raise ValueError("kcache and vcache must be [B, Hkv, Lcap, d] matching q")
-    if not (q.dtype == kcache.dtype == vcache.dtype):
-        raise TypeError("q and the caches must share a dtype")
+    _same_dtype((q, "q"), (kcache, "kcache"), (vcache, "vcache"))
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
     _check(lib.jetlong_prefill_chunk(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
@@ -202,8 +219,10 @@ def prefill_ie(q, k, v, out=None, *, w0: int, w_pretrained: int, rope_theta: flo
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
         raise ValueError("k and v must be [B, Hkv, L, d] matching q")
+    _same_dtype((q, "q"), (k, "k"), (v, "v"))
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     lib = load_library()
     need = int(lib.jetlong_prefill_ie_workspace_size(B, Hq, L, d, _dtype_code(q)))
     if workspace is None:
@@ -238,6 +257,9 @@ def prefill_streamed(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_
     for t, n in ((k_dev, "k_dev"), (v_dev, "v_dev"), (v_host, "v_host")):
         if t.shape != k_host.shape or t.dtype != k_host.dtype:
             raise ValueError(f"{n} must match k_host's shape and dtype")
+    if k_host.shape[0] != B or k_host.shape[2] != L or k_host.shape[3] != d:
+        raise ValueError("k_host must be [B, Hkv, L, d] matching q_host")
+    _same_dtype((q_host, "q_host"), (k_host, "k_host"))
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
     _check(lib.jetlong_prefill_streamed(_host(q_host, "q_host"), _host(k_host, "k_host"),
@@ -261,13 +283,13 @@ def prefill_varlen(q, k, v, lens, out=None, *, w0: int, w_pretrained: int, rope_
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, Lmax, d) or v.shape != k.shape:
         raise ValueError("k and v must be [B, Hkv, Lmax, d] matching q")
-    if not (q.dtype == k.dtype == v.dtype):
-        raise TypeError("q, k, v must share a dtype")
+    _same_dtype((q, "q"), (k, "k"), (v, "v"))
     lens = _np.ascontiguousarray(_np.asarray(lens, dtype=_np.int32).reshape(-1))
     if lens.shape[0] != B:
         raise ValueError("lens must have one length per sequence")
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     lse = torch.empty((B, Hq, Lmax), dtype=torch.float32, device=q.device) if with_lse else None
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
@@ -277,6 +299,16 @@ def prefill_varlen(q, k, v, lens, out=None, *, w0: int, w_pretrained: int, rope_
                                       float(rope_theta), float(scale), _dtype_code(q),
                                       _stream(stream)), lib)
     return (out, lse) if with_lse else out
+
+
+def _decode_shapes(q, kcache, vcache):
+    if q.dim() != 3 or kcache.dim() != 4:
+        raise ValueError("q must be [B, Hq, d] and the caches [B, Hkv, Lcap, d]")
+    if vcache.shape != kcache.shape:
+        raise ValueError("kcache and vcache must have the same shape")
+    if kcache.shape[0] != q.shape[0] or kcache.shape[3] != q.shape[2]:
+        raise ValueError("the caches must be [B, Hkv, Lcap, d] with q's B and d")
+    _same_dtype((q, "q"), (kcache, "kcache"), (vcache, "vcache"))
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, Lcap: int, d: int) -> int:
@@ -297,12 +329,12 @@ def decode(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained: int,
            _entry: str = "jetlong_decode"):
     """One decode step: raw q [B,Hq,d] at position L-1 over cache rows [0, L)."""
     import torch
+    _decode_shapes(q, kcache, vcache)
     B, Hq, d = q.shape
     _, Hkv, Lcap, _ = kcache.shape
-    if vcache.shape != kcache.shape:
-        raise ValueError("kcache and vcache must have the same shape")
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     need = decode_workspace_size(B, Hq, Hkv, Lcap, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -331,12 +363,12 @@ def decode_noalloc(q, kcache, vcache, L: int, out=None, *, w0: int, w_pretrained
     JetLongError(INVALID_ARG).
     """
     import torch
+    _decode_shapes(q, kcache, vcache)
     B, Hq, d = q.shape
     _, Hkv, Lcap, _ = kcache.shape
-    if vcache.shape != kcache.shape:
-        raise ValueError("kcache and vcache must have the same shape")
     if out is None:
         out = torch.empty_like(q)
+    _like(out, q, "out", "q")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     lib = load_library()
     _check(lib.jetlong_decode_noalloc(_dev(q, "q"), _dev(kcache, "kcache"), _dev(vcache, "vcache"),
