@@ -28,8 +28,10 @@
  *     path for prefill) or JETLONG_FP32 (all fp32; CUDA-core fp32 path).
  *     Accumulation is fp32 in both.
  *   - All pointers named d_* or tensor pointers are DEVICE memory owned by the
- *     caller.  The library never writes q, k, v or the caches and allocates no
- *     device memory in any call.
+ *     caller (jetlong_prefill_streamed also takes host buffers, named *_host).
+ *     The library never writes q, k, v or the caches (jetlong_prefill_streamed
+ *     fills the device staging buffers it is given) and allocates no device
+ *     memory in any call.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) on the current device.
  *   - Errors: every entry point returning int returns a jetlong_status.
@@ -119,7 +121,7 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
  * the two forms.  Arguments as jetlong_prefill, plus a device workspace of at
  * least jetlong_prefill_ie_workspace_size(B, Hq, L, d, dtype) bytes (16-byte
  * aligned, caller-owned; the three pass outputs and their LSEs).  Four
- * launches (one when w0 = 0: pass B alone). */
+ * launches; when w0 = 0, pass B alone and a device-to-device copy into out. */
 size_t jetlong_prefill_ie_workspace_size(int B, int Hq, int L, int d, jetlong_dtype dtype);
 int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
                        int B, int Hq, int Hkv, int L, int d,
