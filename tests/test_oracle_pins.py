@@ -334,6 +334,19 @@ MUTANTS = {
     "rope_cache_moved_to_fj": ("if (c->rope_cache) unrotate_cached(c, kraw, kr, j - fj);",
                                "if (c->rope_cache) rotate_cached(c, kraw, kr, fj);"),
     "lse_without_max": ("if (lse) *lse = mx + log(sum);", "if (lse) *lse = log(sum);"),
+    "local_query_aliased": ("            else rotate_cached(c, kraw, kr, j);\n            qq = qe;",
+                            "            else rotate_cached(c, kraw, kr, j);\n            qq = qm;"),
+    "scale_dropped": ("logit[j] = c->scale * a;", "logit[j] = a;"),
+    "decode_query_at_L_minus_2": ("rows[3 * r + 1] = h; rows[3 * r + 2] = L - 1;",
+                                  "rows[3 * r + 1] = h; rows[3 * r + 2] = L - 2;"),
+    "prefill_G_from_L_minus_1": ("J.c.G = jlo_group_size(L, w_pretrained);\n    J.c.scale = scale; "
+                                 "J.c.in_dtype = in_dtype; J.c.npos = L;\n",
+                                 "J.c.G = jlo_group_size(L - 1, w_pretrained);\n    J.c.scale = scale; "
+                                 "J.c.in_dtype = in_dtype; J.c.npos = L;\n"),
+    "decode_G_from_Lcap": ("J.c.G = jlo_group_size(L, w_pretrained);\n    J.c.scale = scale; J.c.in_dtype = in_dtype; "
+                           "J.c.npos = L; J.c.rope_cache = rope_cache;",
+                           "J.c.G = jlo_group_size(Lcap, w_pretrained);\n    J.c.scale = scale; J.c.in_dtype = in_dtype; "
+                           "J.c.npos = L; J.c.rope_cache = rope_cache;"),
     "dropped_self_key": ("for (int64_t j = 0; j <= i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
                          "        for (int t = 0; t < d; ++t) kraw[t]",
                          "for (int64_t j = 0; j < i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
