@@ -1,0 +1,83 @@
+"""CPU checks of the bench's bookkeeping: the tile and FLOP counts that turn
+kernel time into TFLOP/s (against brute force over the (query, key) pairs),
+and the JSON line of the CPU-oracle arm (`--impl reference`)."""
+import io
+import json
+import types
+from contextlib import redirect_stdout
+
+import numpy as np
+import pytest
+
+import bench
+from rope_context_extension_jet_b200 import inputs as I
+
+
+def brute_tiles(L, w0, P=0, bm=128, bn=128):
+    """Causal tiles and tiles holding both local (i - j < w0) and remote causal
+    pairs, by listing every pair of every tile of query rows [P, L)."""
+    tiles = band = 0
+    for i0 in range(P, L, bm):
+        i = np.arange(i0, min(i0 + bm, L))
+        for j0 in range(0, int(i[-1]) + 1, bn):
+            j = np.arange(j0, j0 + bn)
+            diff = i[:, None] - j[None, :]
+            causal = (diff >= 0) & (j[None, :] < L)
+            if not causal.any():
+                continue
+            tiles += 1
+            local = causal & (diff < w0)
+            if local.any() and (causal & ~local).any():
+                band += 1
+    return tiles, band
+
+
+@pytest.mark.parametrize("L,w0,P", [(700, 200, 0), (1000, 1, 0), (1000, 0, 0), (513, 513, 0),
+                                    (1300, 300, 640), (1300, 129, 1200), (257, 128, 0)])
+def test_tile_counts_match_brute_force(L, w0, P):
+    assert bench.tile_counts(L, w0, P=P) == brute_tiles(L, w0, P=P)
+
+
+def test_headline_tile_counts():
+    # 128K, w0 = 4096, 128 x 128 tiles: 1024 query blocks, 524,800 causal tiles,
+    # the band i - j = 4096 crossing 992 of them
+    assert bench.tile_counts(131072, 4096) == (524800, 992)
+
+
+def test_prefill_flops_against_row_sums():
+    w = I.PrefillWorkload("t", 1, "bf16", 2, 4, 2, 64, 1300, 500, 300, 1e4)
+    for P in (0, 640):
+        useful, computed, tiles, band = bench.prefill_flops(w, P=P)
+        rows = np.arange(P, w.L, dtype=np.float64)
+        # QK^T and P.V: 2 * d FLOPs each per causal (i, j) pair, j in [0, i]
+        assert useful == pytest.approx(float(np.sum(4.0 * w.d * (rows + 1))) * w.Hq * w.B, rel=1e-12)
+        # every causal tile computes a full 128 x 128 QK^T and P.V, band tiles one more QK^T
+        assert computed == w.B * w.Hq * (tiles * 4.0 + band * 2.0) * w.d * 128 * 128
+        assert computed >= useful
+
+
+def test_reference_arm_json_line(monkeypatch):
+    real = bench.oracle_prefill_sample
+    monkeypatch.setattr(bench, "oracle_prefill_sample", lambda w, budget_s: real(w, budget_s=0.3))
+    args = types.SimpleNamespace(gpus=1, steps=1, warmup=3)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(args, 0, 1)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == I.C4.name and line["config"]["G"] == 4
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(types.SimpleNamespace(gpus=2, steps=1, warmup=3), 1, 2)
+    assert buf.getvalue() == ""
