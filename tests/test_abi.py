@@ -181,3 +181,43 @@ def test_prefill_ie_workspace_and_arguments(lib):
     args[5] = 3
     assert lib.jetlong_prefill_ie(*args, P, 1 << 30, NULL) == 1             # Hq % Hkv
     assert jl.launch_count() == before
+
+
+def _streamed(lib, **kw):
+    a = dict(qh=P, kh=P, vh=P, oh=P, qd=P, kd=P, vd=P, od=P, B=1, Hq=4, Hkv=2, L=300, d=128, w0=8,
+             wp=32, theta=1e6, scale=0.088, dtype=0, nch=4)
+    a.update(kw)
+    return lib.jetlong_prefill_streamed(a["qh"], a["kh"], a["vh"], a["oh"], a["qd"], a["kd"], a["vd"],
+                                        a["od"], a["B"], a["Hq"], a["Hkv"], a["L"], a["d"], a["w0"],
+                                        a["wp"], a["theta"], a["scale"], a["dtype"], a["nch"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qh=NULL), 1), (dict(oh=NULL), 1), (dict(kd=NULL), 1), (dict(od=NULL), 1), (dict(L=0), 1),
+    (dict(nch=0), 1), (dict(Hkv=3), 1), (dict(d=96), 2), (dict(theta=0.5), 1), (dict(dtype=5), 1),
+])
+def test_prefill_streamed_rejects_bad_arguments_on_host(lib, kw, status):
+    before = jl.launch_count()
+    assert _streamed(lib, **kw) == status
+    assert jl.launch_count() == before
+    assert jl.last_error() != ""
+
+
+def _noalloc(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, B=2, Hq=8, Hkv=2, L=100, Lcap=128, d=128, w0=8, wp=32,
+             theta=1e6, scale=0.088, dtype=0)
+    a.update(kw)
+    return lib.jetlong_decode_noalloc(a["q"], a["kc"], a["vc"], a["out"], a["B"], a["Hq"], a["Hkv"],
+                                      a["L"], a["Lcap"], a["d"], a["w0"], a["wp"], a["theta"],
+                                      a["scale"], a["dtype"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=NULL), 1), (dict(vc=ctypes.c_void_p((1 << 20) + 8)), 1), (dict(L=0), 1),
+    (dict(L=129), 1), (dict(Hkv=3), 1), (dict(d=80), 2), (dict(wp=0), 1), (dict(scale=float("nan")), 1),
+])
+def test_decode_noalloc_rejects_bad_arguments_on_host(lib, kw, status):
+    before = jl.launch_count()
+    assert _noalloc(lib, **kw) == status
+    assert jl.launch_count() == before
+    assert jl.last_error() != ""
