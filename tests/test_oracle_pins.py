@@ -173,7 +173,10 @@ def pin_reduction_zero_window(lib):
 
 def pin_inclusion_exclusion(lib):
     # the pages' three-pass LSE merge reaches the same routed output
-    for L, w0, w_pre in ((64, 8, 16), (64, 1, 20), (50, 13, 11), (37, 36, 5), (64, 63, 30)):
+    # w0 = 0: the window passes are empty (LSE -inf, weight 0) and B alone remains;
+    # w0 >= L: C equals B and cancels, A alone remains
+    for L, w0, w_pre in ((64, 8, 16), (64, 1, 20), (50, 13, 11), (37, 36, 5), (64, 63, 30),
+                         (40, 0, 9), (40, 40, 9), (33, 1000, 7)):
         G = -(-L // w_pre)
         out, q, k, v, sc = _prefill_small(lib, L, w0, w_pre, seed=L + w0)
         ref = tb.inclusion_exclusion(q, k, v, w0, G, 1e4, sc)
