@@ -134,10 +134,11 @@ def pin_routing_enumeration(lib):
         assert local == sum(min(i + 1, w0) for i in range(L)), (L, w0, local)
 
 
-def _prefill_small(lib, L, w0, w_pre, Hq=4, Hkv=2, d=16, theta=1e4, seed=0, dtype="fp32"):
-    q = _rand((1, Hq, L, d), seed)
-    k = _rand((1, Hkv, L, d), seed + 1)
-    v = _rand((1, Hkv, L, d), seed + 2)
+def _prefill_small(lib, L, w0, w_pre, Hq=4, Hkv=2, d=16, theta=1e4, seed=0, dtype="fp32", B=2):
+    # two sequences, so the per-sequence offsets of q, k, v and out are pinned too
+    q = _rand((B, Hq, L, d), seed)
+    k = _rand((B, Hkv, L, d), seed + 1)
+    v = _rand((B, Hkv, L, d), seed + 2)
     scale = 1.0 / math.sqrt(d)
     out = oracle.prefill(q, k, v, w0=w0, w_pretrained=w_pre, rope_theta=theta, scale=scale,
                          nthreads=2, lib=lib)
@@ -184,23 +185,23 @@ def pin_inclusion_exclusion(lib):
 
 
 def pin_decode_matches_prefill_row(lib):
-    L, Hq, Hkv, d, w0, w_pre = 45, 4, 2, 16, 6, 10
-    q = _rand((1, Hq, L, d), 21)
-    k = _rand((1, Hkv, L, d), 22)
-    v = _rand((1, Hkv, L, d), 23)
+    B, L, Hq, Hkv, d, w0, w_pre = 2, 45, 4, 2, 16, 6, 10
+    q = _rand((B, Hq, L, d), 21)
+    k = _rand((B, Hkv, L, d), 22)
+    v = _rand((B, Hkv, L, d), 23)
     sc = 0.25
-    rows = np.array([(0, h, L - 1) for h in range(Hq)], dtype=np.int32)
+    rows = np.array([(b, h, L - 1) for b in range(B) for h in range(Hq)], dtype=np.int32)
     pre = oracle.prefill_rows(q, k, v, rows, w0=w0, w_pretrained=w_pre, rope_theta=1e4, scale=sc,
                               lib=lib)
     Lcap = L + 7
-    kc = np.zeros((1, Hkv, Lcap, d), np.float32)
-    vc = np.zeros((1, Hkv, Lcap, d), np.float32)
+    kc = np.zeros((B, Hkv, Lcap, d), np.float32)
+    vc = np.zeros((B, Hkv, Lcap, d), np.float32)
     kc[:, :, :L] = k
     vc[:, :, :L] = v
     kc[:, :, L:] = 1e3  # rows past L must be ignored
     dec = oracle.decode(np.ascontiguousarray(q[:, :, L - 1]), kc, vc, L, w0=w0, w_pretrained=w_pre,
                         rope_theta=1e4, scale=sc, lib=lib)
-    np.testing.assert_allclose(dec[0], pre, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dec.reshape(B * Hq, d), pre, rtol=0, atol=1e-13)
 
 
 def pin_row_lse_textbook(lib):
@@ -350,6 +351,12 @@ MUTANTS = {
                            "J.c.npos = L; J.c.rope_cache = rope_cache;",
                            "J.c.G = jlo_group_size(Lcap, w_pretrained);\n    J.c.scale = scale; J.c.in_dtype = in_dtype; "
                            "J.c.npos = L; J.c.rope_cache = rope_cache;"),
+    "decode_query_of_sequence_0": ("size_t q_off = J->q_is_decode ? ((size_t)b * J->Hq + h) * d",
+                                   "size_t q_off = J->q_is_decode ? ((size_t)0 * J->Hq + h) * d"),
+    "prefill_query_of_sequence_0": (": (((size_t)b * J->Hq + h) * J->L + i) * d;",
+                                    ": (((size_t)0 * J->Hq + h) * J->L + i) * d;"),
+    "keys_of_sequence_0": ("size_t kv_off = ((size_t)b * J->Hkv + kvh) * (size_t)J->Lkv * d;",
+                           "size_t kv_off = ((size_t)0 * J->Hkv + kvh) * (size_t)J->Lkv * d;"),
     "dropped_self_key": ("for (int64_t j = 0; j <= i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
                          "        for (int t = 0; t < d; ++t) kraw[t]",
                          "for (int64_t j = 0; j < i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
