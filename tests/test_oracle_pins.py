@@ -279,12 +279,26 @@ def pin_rope_cache_decode_composition(lib):
         np.testing.assert_allclose(a, b, rtol=0, atol=2e-5)
 
 
+def pin_bf16_widening(lib):
+    # bf16 inputs are the upper 16 bits of an fp32: the oracle on bf16 bits equals
+    # the oracle on those values given as fp32 (numpy's own view of the bits)
+    from rope_context_extension_jet_b200.inputs import bf16_bits_to_f32, to_bf16_bits
+    L, d = 40, 16
+    qb = to_bf16_bits(_rand((1, 2, L, d), 1))
+    kb = to_bf16_bits(_rand((1, 2, L, d), 2))
+    vb = to_bf16_bits(_rand((1, 2, L, d), 3))
+    kw = dict(w0=5, w_pretrained=16, rope_theta=1e4, scale=0.25, lib=lib)
+    a = oracle.prefill(qb, kb, vb, **kw)
+    b = oracle.prefill(bf16_bits_to_f32(qb), bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), **kw)
+    np.testing.assert_array_equal(a, b)
+
+
 PINS = [pin_group_size_table, pin_remote_position, pin_rotation_closed_form,
         pin_rotation_algebra, pin_relative_invariance, pin_routing_enumeration,
         pin_reduction_g1, pin_reduction_wide_window, pin_reduction_zero_window,
         pin_inclusion_exclusion, pin_decode_matches_prefill_row, pin_row_lse_textbook,
         pin_rotate_rows_textbook,
-        pin_rope_cache_decode_textbook, pin_rope_cache_decode_composition]
+        pin_rope_cache_decode_textbook, pin_rope_cache_decode_composition, pin_bf16_widening]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -292,16 +306,6 @@ def test_oracle_pin(pin):
     pin(oracle.load())
 
 
-def test_bf16_inputs_widen_exactly():
-    from rope_context_extension_jet_b200.inputs import bf16_bits_to_f32, to_bf16_bits
-    L, d = 40, 16
-    qb = to_bf16_bits(_rand((1, 2, L, d), 1))
-    kb = to_bf16_bits(_rand((1, 2, L, d), 2))
-    vb = to_bf16_bits(_rand((1, 2, L, d), 3))
-    kw = dict(w0=5, w_pretrained=16, rope_theta=1e4, scale=0.25)
-    a = oracle.prefill(qb, kb, vb, **kw)
-    b = oracle.prefill(bf16_bits_to_f32(qb), bf16_bits_to_f32(kb), bf16_bits_to_f32(vb), **kw)
-    np.testing.assert_array_equal(a, b)
 
 
 def test_bf16_rounding_is_nearest_even():
@@ -357,6 +361,8 @@ MUTANTS = {
                                     ": (((size_t)0 * J->Hq + h) * J->L + i) * d;"),
     "keys_of_sequence_0": ("size_t kv_off = ((size_t)b * J->Hkv + kvh) * (size_t)J->Lkv * d;",
                            "size_t kv_off = ((size_t)0 * J->Hkv + kvh) * (size_t)J->Lkv * d;"),
+    "bf16_widened_one_bit_low": ("uint32_t bits = ((uint32_t)((const uint16_t*)base)[idx]) << 16;",
+                                 "uint32_t bits = ((uint32_t)((const uint16_t*)base)[idx]) << 15;"),
     "dropped_self_key": ("for (int64_t j = 0; j <= i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
                          "        for (int t = 0; t < d; ++t) kraw[t]",
                          "for (int64_t j = 0; j < i; ++j) {\n        size_t off = kv_off + (size_t)j * d;\n"
