@@ -193,18 +193,61 @@ static void attend_row(const row_ctx* c, const void* q, size_t q_off,
     if (lse) *lse = mx + log(sum);
 }
 
-static double* build_cs(int d, int64_t npos, double rope_theta)
+/* cos/sin of p * theta_m for positions [0, npos): the same libm values as
+ * jlo_rotate computes for each position (theta_m evaluated once per m, the
+ * product and cos/sin once per (p, m)).  Filled by the host's threads over
+ * disjoint position ranges; each entry is computed exactly as a serial loop
+ * would compute it. */
+typedef struct {
+    double* cs;
+    const double* freq;
+    int h;
+    int64_t p0, p1;
+} cs_part;
+
+static void* fill_cs(void* arg)
+{
+    cs_part* P = (cs_part*)arg;
+    for (int64_t p = P->p0; p < P->p1; ++p)
+        for (int m = 0; m < P->h; ++m) {
+            double phi = (double)p * P->freq[m];
+            P->cs[((size_t)p * P->h + m) * 2] = cos(phi);
+            P->cs[((size_t)p * P->h + m) * 2 + 1] = sin(phi);
+        }
+    return NULL;
+}
+
+static double* build_cs_threads(int d, int64_t npos, double rope_theta, int nthreads)
 {
     int h = d / 2;
-    double* cs = (double*)malloc(sizeof(double) * 2 * (size_t)h * (size_t)npos);
+    double freq[256];
+    for (int m = 0; m < h; ++m) freq[m] = inv_freq(m, d, rope_theta);
+    double* cs = (double*)malloc(sizeof(double) * 2 * (size_t)h * (size_t)(npos > 0 ? npos : 1));
     if (!cs) return NULL;
-    for (int64_t p = 0; p < npos; ++p)
-        for (int m = 0; m < h; ++m) {
-            double phi = (double)p * inv_freq(m, d, rope_theta);
-            cs[((size_t)p * h + m) * 2] = cos(phi);
-            cs[((size_t)p * h + m) * 2 + 1] = sin(phi);
-        }
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if ((int64_t)nthreads * 1024 > npos) nthreads = (int)(npos / 1024) + 1;
+    cs_part part[256];
+    pthread_t th[256];
+    int started[256] = {0};
+    for (int t = 0; t < nthreads; ++t) {
+        part[t].cs = cs; part[t].freq = freq; part[t].h = h;
+        part[t].p0 = npos * t / nthreads;
+        part[t].p1 = npos * (t + 1) / nthreads;
+    }
+    for (int t = 1; t < nthreads; ++t) started[t] = pthread_create(&th[t], NULL, fill_cs, &part[t]) == 0;
+    fill_cs(&part[0]);
+    for (int t = 1; t < nthreads; ++t) {
+        if (started[t]) pthread_join(th[t], NULL);
+        else fill_cs(&part[t]);
+    }
     return cs;
+}
+
+static double* build_cs(int d, int64_t npos, double rope_theta)
+{
+    return build_cs_threads(d, npos, rope_theta, 0);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -300,11 +343,16 @@ int jlo_prefill_rows_lse(const void* q, const void* k, const void* v, int in_dty
         if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 || rows[3 * r + 1] >= Hq ||
             rows[3 * r + 2] < 0 || rows[3 * r + 2] >= L)
             return -1;
+    /* every position a row reaches (i, j <= i and their aliases) is <= the
+     * largest query position asked for */
+    int64_t npos = 1;
+    for (int64_t r = 0; r < n; ++r)
+        if ((int64_t)rows[3 * r + 2] + 1 > npos) npos = (int64_t)rows[3 * r + 2] + 1;
     job_t J;
     memset(&J, 0, sizeof J);
     J.c.d = d; J.c.w0 = w0; J.c.G = jlo_group_size(L, w_pretrained);
-    J.c.scale = scale; J.c.in_dtype = in_dtype; J.c.npos = L;
-    J.c.cs = build_cs(d, L, rope_theta);
+    J.c.scale = scale; J.c.in_dtype = in_dtype; J.c.npos = npos;
+    J.c.cs = build_cs_threads(d, npos, rope_theta, nthreads);
     if (!J.c.cs) return -2;
     J.q = q; J.k = k; J.v = v; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.L = L; J.Lkv = L;
     J.rows = rows; J.n = n; J.out = out; J.lse = lse;
@@ -383,7 +431,7 @@ static int decode_impl(const void* q, const void* kcache, const void* vcache, in
     memset(&J, 0, sizeof J);
     J.c.d = d; J.c.w0 = w0; J.c.G = jlo_group_size(L, w_pretrained);
     J.c.scale = scale; J.c.in_dtype = in_dtype; J.c.npos = L; J.c.rope_cache = rope_cache;
-    J.c.cs = build_cs(d, L, rope_theta);
+    J.c.cs = build_cs_threads(d, L, rope_theta, nthreads);
     if (!J.c.cs) { free(rows); return -2; }
     J.q = q; J.k = kcache; J.v = vcache; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.L = L; J.Lkv = Lcap;
     J.q_is_decode = 1; J.rows = rows; J.n = n; J.out = out;

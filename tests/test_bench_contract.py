@@ -58,7 +58,8 @@ def test_prefill_flops_against_row_sums():
 
 def test_reference_arm_json_line(monkeypatch):
     real = bench.oracle_prefill_sample
-    monkeypatch.setattr(bench, "oracle_prefill_sample", lambda w, budget_s: real(w, budget_s=0.3))
+    monkeypatch.setattr(bench, "oracle_prefill_sample",
+                        lambda w, budget_s, **kw: real(w, budget_s=0.3, **kw))
     args = types.SimpleNamespace(gpus=1, steps=1, warmup=3)
     buf = io.StringIO()
     with redirect_stdout(buf):
@@ -81,3 +82,21 @@ def test_reference_arm_other_ranks_print_nothing():
     with redirect_stdout(buf):
         bench.run_reference(types.SimpleNamespace(gpus=2, steps=1, warmup=3), 1, 2)
     assert buf.getvalue() == ""
+
+
+def test_per_clock_figures():
+    # 900.8 TFLOP/s at an 1852 MHz SM clock: 486.4 TFLOP/s per GHz, and 40.1% of
+    # the tensor pipe's 148 SMs x 8192 FLOP/cycle at that clock
+    peaks = {"bf16_tflops_sustained": 1401.4, "bf16_sustained_sm_mhz": 1335.0}
+    r = bench.per_clock(900.8, 1852.0, peaks)
+    assert r["tflops_per_ghz"] == pytest.approx(486.39, abs=0.01)
+    assert r["frac_of_tensor_pipe_at_this_clock"] == pytest.approx(900.8e12 / (148 * 8192 * 1852e6), abs=1e-4)
+    assert r["sustained_peak_tflops_per_ghz"] == pytest.approx(1401.4 / 1.335, abs=0.01)
+    assert r["frac_of_sustained_peak_per_clock"] == pytest.approx(486.39 / (1401.4 / 1.335), abs=1e-3)
+    assert bench.per_clock(900.8, None, peaks) is None
+
+
+def test_peak_clock_lookup_searches_nested_keys():
+    d = {"hbm_gbs": 6548.5, "bf16": {"sustained": {"sm_mhz_median_sustained": 1335}, "burst_sm_mhz": 1900},
+         "mem_clock_mhz_sustained": 3996}
+    assert bench._find_mhz(d, "sustain") == 1335.0

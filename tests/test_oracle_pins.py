@@ -348,9 +348,9 @@ MUTANTS = {
     "decode_query_at_L_minus_2": ("rows[3 * r + 1] = h; rows[3 * r + 2] = L - 1;",
                                   "rows[3 * r + 1] = h; rows[3 * r + 2] = L - 2;"),
     "prefill_G_from_L_minus_1": ("J.c.G = jlo_group_size(L, w_pretrained);\n    J.c.scale = scale; "
-                                 "J.c.in_dtype = in_dtype; J.c.npos = L;\n",
+                                 "J.c.in_dtype = in_dtype; J.c.npos = npos;\n",
                                  "J.c.G = jlo_group_size(L - 1, w_pretrained);\n    J.c.scale = scale; "
-                                 "J.c.in_dtype = in_dtype; J.c.npos = L;\n"),
+                                 "J.c.in_dtype = in_dtype; J.c.npos = npos;\n"),
     "decode_G_from_Lcap": ("J.c.G = jlo_group_size(L, w_pretrained);\n    J.c.scale = scale; J.c.in_dtype = in_dtype; "
                            "J.c.npos = L; J.c.rope_cache = rope_cache;",
                            "J.c.G = jlo_group_size(Lcap, w_pretrained);\n    J.c.scale = scale; J.c.in_dtype = in_dtype; "
