@@ -330,6 +330,163 @@ def run_profile(args):
     print(json.dumps({"profile": args.profile, "L": args.L, "launches": jl.launch_count()}))
 
 
+# ---------------------------------------------------------------- ncu harness
+# Counters read for one kernel launch (a few replay passes; run on the reduced
+# --profile workloads only).
+NCU_METRICS = (
+    "gpu__time_duration.sum",
+    "sm__cycles_elapsed.avg.per_second",
+    "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active",
+    "smsp__issue_active.avg.pct_of_peak_sustained_active",
+    "sm__inst_executed_pipe_xu.avg.pct_of_peak_sustained_active",
+    "sm__warps_active.avg.pct_of_peak_sustained_active",
+    "dram__bytes_read.sum",
+    "dram__bytes_write.sum",
+    "gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed",
+    "launch__registers_per_thread",
+    "smsp__inst_executed.sum",
+)
+NCU_KERNELS = {"prefill": "prefill_pair_kernel", "decode": "decode_tc_kernel"}
+
+
+def parse_ncu_csv(text):
+    """Rows of ncu's --csv metric output as dicts {kernel, id, metric, unit, value}."""
+    import csv
+    import io
+    lines = [ln for ln in text.splitlines() if ln.startswith('"')]
+    rows = []
+    for r in csv.DictReader(io.StringIO("\n".join(lines))):
+        try:
+            val = float(r["Metric Value"].replace(",", ""))
+        except (KeyError, ValueError):
+            continue
+        rows.append({"kernel": r.get("Kernel Name", ""), "id": int(r.get("ID", 0)),
+                     "metric": r["Metric Name"], "unit": r.get("Metric Unit", ""), "value": val})
+    return rows
+
+
+def launch_summary(rows):
+    """Per kernel (name up to its template arguments): launches, total ms, share
+    of the summed device time, from gpu__time_duration.sum rows (ns)."""
+    per = {}
+    for r in rows:
+        if r["metric"] != "gpu__time_duration.sum":
+            continue
+        name = r["kernel"].split("(")[0].strip()
+        n, t = per.get(name, (0, 0.0))
+        per[name] = (n + 1, t + r["value"] * 1e-6)
+    total = sum(t for _, t in per.values()) or 1.0
+    return sorted(((k, n, t, t / total) for k, (n, t) in per.items()), key=lambda x: -x[2])
+
+
+def _ncu_cmd(extra, bench_args, log):
+    return (["ncu", "--clock-control", "none", "--print-units", "base", "--csv", "--log-file", log] + extra
+            + [sys.executable, os.path.join(ROOT, "bench.py")] + bench_args)
+
+
+def run_ncu(args):
+    """Profiling harness: run the bench command once without ncu (it must exit 0),
+    then the same command under ncu, and write the summary under profiles/."""
+    out_dir = os.path.join(ROOT, "gpurun_out")
+    os.makedirs(out_dir, exist_ok=True)
+    peaks = load_peaks()
+    if args.ncu == "launches":
+        bench_args = ["--steps", str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
+        extra = ["--metrics", "gpu__time_duration.sum"]
+    elif args.ncu == "traffic":
+        bench_args = ["--profile", "prefill", "--L", str(args.L), "--steps", "1", "--warmup", "1"]
+        extra = ["--metrics", "gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum",
+                 "-k", "regex:" + NCU_KERNELS["prefill"], "-s", "1", "-c", "1"]
+    else:
+        bench_args = ["--profile", args.ncu, "--L", str(args.L), "--steps", "1", "--warmup", "1"]
+        extra = ["--metrics", ",".join(NCU_METRICS), "-k", "regex:" + NCU_KERNELS[args.ncu], "-s", "1", "-c", "1"]
+    plain = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + bench_args,
+                           capture_output=True, text=True)
+    if plain.returncode != 0:
+        print(plain.stdout[-2000:], plain.stderr[-2000:])
+        raise SystemExit(f"plain run exited {plain.returncode}; not profiling")
+    log = os.path.join(out_dir, f"ncu_{args.ncu}.csv")
+    cmd = _ncu_cmd(extra, bench_args, log)
+    t0 = time.time()
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    secs = time.time() - t0
+    if r.returncode != 0:
+        print(r.stdout[-2000:], r.stderr[-2000:])
+        raise SystemExit(f"ncu exited {r.returncode}")
+    rows = parse_ncu_csv(open(log).read())
+    shown = " ".join(("'" + c + "'") if ("(" in c or " " in c) else c
+                     for c in ["ncu"] + cmd[1:4] + cmd[6:] if c != sys.executable).replace(
+        os.path.join(ROOT, ""), "")
+    shown = shown.replace(" bench.py", " python bench.py").replace("--log-file", "")
+    lines = []
+    if args.ncu == "launches":
+        summ = launch_summary(rows)
+        lines += [f"# Launch list: `python bench.py {' '.join(bench_args)}`", "",
+                  "Every launch of the bench command with its device time (ncu, one pass, serialised and",
+                  "cold-cache: compare shares, not absolute times).", "", "Command (run after the same bench",
+                  "command exited 0 without ncu):", "", "    " + shown, "",
+                  "| kernel | launches | total ms | share |", "|---|---|---|---|"]
+        lines += [f"| `{k}` | {n} | {t:.3f} | {sh:.1%} |" for k, n, t, sh in summ]
+        rec = {"launches": [{"kernel": k, "launches": n, "total_ms": round(t, 4), "share": round(sh, 4)}
+                            for k, n, t, sh in summ]}
+        name = "launches_bench"
+    else:
+        m = {r["metric"]: r["value"] for r in rows}
+        dur = m.get("gpu__time_duration.sum", float("nan")) * 1e-9
+        dram = m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0)
+        rec = {"metrics": m, "seconds": dur, "dram_bytes": dram}
+        if args.ncu in ("prefill", "traffic"):
+            w = I.C4.with_(L=args.L)
+            useful, computed, _, _ = prefill_flops(w)
+            rec.update({"workload": f"prefill bf16 B=1 Hq=32 Hkv=8 d=128 L={args.L} G={max(1, -(-args.L // w.w_pretrained))} "
+                                    f"w0={w.w0}", "flops_computed": computed,
+                        "tflops": computed / dur / 1e12 if dur > 0 else None})
+            rec["frac_of_bf16_burst"] = rec["tflops"] / peaks["bf16_tflops"] if rec["tflops"] else None
+            kname = NCU_KERNELS["prefill"]
+        else:
+            w = I.D.with_(L0=args.L - 1, Lcap=args.L + 64, steps=1)
+            kv, allb = decode_bytes(w, args.L)
+            rec.update({"workload": f"decode bf16 B=8 Hq=32 Hkv=8 d=128 L={args.L}", "kv_bytes": kv,
+                        "gbs_kv": kv / dur / 1e9 if dur > 0 else None})
+            rec["frac_of_hbm"] = rec["gbs_kv"] / peaks["hbm_gbs"] if rec["gbs_kv"] else None
+            kname = NCU_KERNELS["decode"]
+        rec["peaks"] = {k: v for k, v in peaks.items()}
+        if args.ncu == "traffic":
+            name = f"{kname}_L{args.L}_dram"
+        else:
+            name = f"{kname}_L{args.L}_counters"
+        lines += [f"# `{kname}`: {rec['workload']}", "", "One launch after one warm-up launch (ncu, clock control none),",
+                  "captured after the same command exited 0 without ncu:", "", "    " + shown, "",
+                  "| metric | value |", "|---|---|"]
+        lines += [f"| `{k}` | {v:.6g} |" for k, v in m.items()]
+        if "tflops" in rec:
+            lines += ["", f"Computed FLOPs {rec['flops_computed']:.4e} over {dur * 1e3:.3f} ms = "
+                          f"{rec['tflops']:.1f} TFLOP/s, {rec['frac_of_bf16_burst']:.3f} of the {peaks['source']} "
+                          f"bf16 burst peak ({peaks['bf16_tflops']} TFLOP/s); DRAM {dram / 1e9:.3f} GB "
+                          f"({dram / dur / 1e9:.0f} GB/s)."]
+        else:
+            lines += ["", f"K/V bytes {rec['kv_bytes']:.4e} over {dur * 1e3:.3f} ms = {rec['gbs_kv']:.0f} GB/s, "
+                          f"{rec['frac_of_hbm']:.3f} of the {peaks['source']} HBM copy bandwidth "
+                          f"({peaks['hbm_gbs']} GB/s); DRAM counted {dram / 1e9:.3f} GB."]
+    lines += ["", f"Sources: sha256 of the prefill kernel files {prefill_source_hash()[:16]}; "
+                  f"capture took {secs:.0f} s."]
+    prof = os.path.join(ROOT, "profiles")
+    with open(os.path.join(prof, name + ".md"), "w") as f:
+        f.write("\n".join(lines) + "\n")
+    if args.ncu == "traffic" and args.L == I.C4.L:
+        tr_path = os.path.join(prof, "traffic.json")
+        try:
+            tr = json.load(open(tr_path))
+        except (OSError, ValueError):
+            tr = {}
+        tr[PREFILL_KERNEL] = {"dram_bytes_per_launch": dram, "source_sha256": prefill_source_hash(),
+                              "workload": rec["workload"], "command": shown}
+        with open(tr_path, "w") as f:
+            json.dump(tr, f, indent=1)
+    print(json.dumps({"ncu": args.ncu, "summary": os.path.join("profiles", name + ".md"),
+                      "seconds": round(secs, 1)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -341,6 +498,10 @@ def main():
     ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
                     help="run only one kernel on a reduced workload (for ncu captures)")
     ap.add_argument("--L", type=int, default=32768, help="sequence / cache length for --profile")
+    ap.add_argument("--ncu", choices=["launches", "prefill", "decode", "traffic"], default=None,
+                    help="profiling harness: the bench command (launches), one kernel of the --profile "
+                         "workloads (prefill, decode) or one full-size prefill's DRAM bytes (traffic, "
+                         "--L 131072), under ncu; writes the summary under profiles/")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -350,6 +511,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.ncu:
+        run_ncu(args)
         return
     if args.profile:
         run_profile(args)

@@ -27,6 +27,16 @@
  *   - Element type: JETLONG_BF16 (q, k, v, caches and out are bf16; tensor-core
  *     path for prefill) or JETLONG_FP32 (all fp32; CUDA-core fp32 path).
  *     Accumulation is fp32 in both.
+ *   - Input range (bf16): q and k may hold any finite bf16 values whose logits
+ *     scale * <q, k> are finite in fp32.  The rotated Q K^T operands are
+ *     rounded to fp16 (11-bit significand) after a power-of-two scaling chosen
+ *     from the data: the prefill scales all queries and all keys of a call so
+ *     the largest of each lies in [2^13, 2^14) (inputs more than 2^27 below the
+ *     largest of their tensor lose relative precision, negligible in any
+ *     logit); the decode scales each query head, and each key row of a key
+ *     block whose unscaled logits would not be finite.  The scales are exact
+ *     and undone in the softmax.  v: |v| below ~1e36 (P.V accumulates in fp32).
+ *     NaN inputs give NaN outputs.
  *   - All pointers named d_* or tensor pointers are DEVICE memory owned by the
  *     caller (jetlong_prefill_streamed also takes host buffers, named *_host).
  *     The library never writes q, k, v or the caches (jetlong_prefill_streamed
@@ -138,7 +148,10 @@ int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
  *   tensors of the same shapes, owned by the caller, 16-byte aligned.
  *   nchunks >= 1; other arguments as jetlong_prefill.
  * Asynchronous: work queued on `stream` afterwards runs after out_host is
- * complete.  Same result as copying in, jetlong_prefill, copying out. */
+ * complete.  Same result as copying in, jetlong_prefill, copying out.  If the
+ * call fails part-way, work queued on `stream` afterwards still runs only
+ * after every copy the call did queue (so the buffers can be freed or reused
+ * in stream order). */
 int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                              void* q_dev, void* k_dev, void* v_dev, void* out_dev,
                              int B, int Hq, int Hkv, int L, int d,
@@ -220,6 +233,30 @@ int jetlong_device_status(void* stream);
  * the word).  No fault, no hang; the context stays usable.  Returns
  * JETLONG_OK or JETLONG_ERR_CUDA (launch failure). */
 int jetlong_selftest_wait_timeout(void* stream);
+
+/* Failure-detection test hook (the pages have no counterpart).  Arms a
+ * one-shot fault injection for the next attention call made on this host
+ * thread: the kernel it launches withholds one barrier arrival, chosen by
+ * `site`, and every bounded wait of that launch gives up after `wait_cycles`
+ * SM cycles instead of the normal ~0.5 s (prefill) / ~2 s (decode).  The
+ * waits that depend on the withheld arrival expire; the kernel records a code
+ * in the device error word, its roles stop, drain their own copies and MMAs,
+ * release tensor memory and return, so the next jetlong_device_status reports
+ * JETLONG_ERR_TIMEOUT and the context stays usable.  The output of the
+ * sabotaged call is undefined.  No fault, trap or unbounded wait is involved.
+ *   JETLONG_INJECT_PREFILL_KEY_TILE: bf16 prefill (both tensor-core kernels):
+ *       the first key tile of every work unit is never released to the MMA
+ *       issuer.
+ *   JETLONG_INJECT_DECODE_COPY: bf16 decode: the first K/V stage of every
+ *       key split is never loaded.
+ * The hook is consumed by the next prefill or decode call of this thread that
+ * passes argument validation (whatever its dtype; the fp32 kernels ignore it);
+ * JETLONG_INJECT_NONE disarms it.  wait_cycles in [1e4, 4e9] (ignored for
+ * JETLONG_INJECT_NONE).  Returns JETLONG_OK or JETLONG_ERR_INVALID_ARG. */
+#define JETLONG_INJECT_NONE 0
+#define JETLONG_INJECT_PREFILL_KEY_TILE 1
+#define JETLONG_INJECT_DECODE_COPY 2
+int jetlong_debug_inject_timeout(int site, long long wait_cycles);
 
 /* Message for the last failing call on this host thread ("" if none). */
 const char* jetlong_last_error(void);

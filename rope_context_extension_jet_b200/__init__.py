@@ -23,7 +23,8 @@ __all__ = [
     "BF16", "FP32", "JetLongError", "load_library", "group_size", "position_map", "prefill",
     "prefill_chunk", "prefill_varlen", "prefill_ie", "prefill_streamed", "decode_workspace_size",
     "decode", "decode_rope_cache", "decode_noalloc", "device_status", "last_error", "launch_count",
-    "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout",
+    "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout", "debug_inject_timeout",
+    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +89,8 @@ def load_library(path: str | None = None):
                                                i32, dbl, flt, i32, vp]
         lib.jetlong_selftest_wait_timeout.restype = i32
         lib.jetlong_selftest_wait_timeout.argtypes = [vp]
+        lib.jetlong_debug_inject_timeout.restype = i32
+        lib.jetlong_debug_inject_timeout.argtypes = [i32, ctypes.c_longlong]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -382,6 +385,20 @@ def selftest_wait_timeout(stream=None):
     """Launch the bounded-wait self test; the next device_status() raises TIMEOUT."""
     lib = load_library()
     _check(lib.jetlong_selftest_wait_timeout(_stream(stream)), lib)
+
+
+# Sites of the failure-detection test hook (JETLONG_INJECT_*).
+INJECT_PREFILL_KEY_TILE = 1
+INJECT_DECODE_COPY = 2
+
+
+def debug_inject_timeout(site: int, wait_cycles: int):
+    """Arm the one-shot test hook: the next prefill or decode call of this thread
+    withholds one barrier arrival (``site``) with every bounded wait limited to
+    ``wait_cycles`` SM cycles, so its waits expire and the following
+    device_status() raises TIMEOUT (jetlong_debug_inject_timeout)."""
+    lib = load_library()
+    _check(lib.jetlong_debug_inject_timeout(int(site), int(wait_cycles)), lib)
 
 
 def device_status(stream=None):

@@ -38,6 +38,8 @@ struct DecodeLaunch {
     float* partials;                 // [B][Hq][n_splits][D + 2]
     unsigned int* tickets;           // [B][Hkv * hgroups]
     int* dev_error;
+    long long wait_cycles;           // limit of every bounded wait
+    int inject;                      // kInjectNone, or the arrival this launch withholds (test hook)
 };
 
 // Unsigned division by the invariant G (Granlund & Montgomery, "Division by
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % STAGES;
-                if (c >= STAGES && !mbar_wait(&empty[st], ((c / STAGES) - 1) & 1)) {
+                if (c >= STAGES && !mbar_wait(&empty[st], ((c / STAGES) - 1) & 1, dl.wait_cycles)) {
                     record_error(dl.dev_error, 0x101);
                     break;
                 }
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
             }
             // drain: every issued copy has landed before the ring is reused / the CTA exits
             for (int c = max(0, issued - STAGES); c < issued; ++c)
-                if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_error(dl.dev_error, 0x102);
+                if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1, dl.wait_cycles)) record_error(dl.dev_error, 0x102);
         }
     } else {
         // ---------------- consumers
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(NT, 2) decode_split_kernel(DecodeProblem p, De
         float qlo[HPB][PPL], qhi[HPB][PPL];
         for (int c = 0; c < nchunks && ok; ++c) {
             const int st = c % STAGES;
-            if (!mbar_wait(&full[st], (c / STAGES) & 1)) {
+            if (!mbar_wait(&full[st], (c / STAGES) & 1, dl.wait_cycles)) {
                 record_error(dl.dev_error, 0x103);
                 ok = false;
                 break;
@@ -399,7 +401,8 @@ struct DecTcCfg {
     static constexpr int PBUF = BIG;                       // [TC_NCW][16 keys][8 heads] bf16
     static constexpr int SQ = PBUF + TC_NCW * 256;         // [2][HPB][D] fp32 rotated queries
     static constexpr int TURNS = SQ + 2 * HPB * D * 4;     // [d/2] uint2 phase constants
-    static constexpr int BARS = TURNS + (D / 2) * 8;
+    static constexpr int QEXP = TURNS + (D / 2) * 8;       // [8] int query exponents, [1] large-query flag
+    static constexpr int BARS = QEXP + 48;
     static constexpr int END = BARS + 2 * TC_STAGES * 8 + 16;
     static constexpr int TOTAL = END + 1024;
 };
@@ -451,41 +454,101 @@ __device__ __forceinline__ uint32_t dec_sw(uint32_t tile, int key, int ch)
     return tile + (uint32_t)((ch >> 3) * (TC_KROWS * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4));
 }
 
+// Operand range of the fp16 Q K^T MMAs.  The rotated keys and queries are
+// rounded to fp16 (11-bit significand, largest value 65504; bf16 inputs reach
+// 3.4e38), so each key row and each query head is first scaled by a power of
+// two that brings its largest |x| into [2^13, 2^14): a rotated value is then
+// below 2^14.5, and powers of two are exact both ways, so multiplying a logit by
+// 2^-(e_q + e_k) gives the logit of the unscaled vectors.  Exponents are clamped
+// to [-100, 100].
+__device__ __forceinline__ uint32_t absmax_bf16x2_dec(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Exponent e with m * 2^e in [2^13, 2^14) for a largest magnitude m given by its
+// bf16 (15-bit) magnitude bits; 0 for zero or a non-finite m.
+__device__ __forceinline__ int range_exp_bf16(uint32_t mag)
+{
+    if (mag == 0u || mag >= 0x7f80u) return 0;
+    const int biased = (int)(mag >> 7);
+    return min(100, max(-100, 13 - ((biased == 0 ? 1 : biased) - 127)));
+}
+
+__device__ __forceinline__ float pow2i_dec(int e) { return __int_as_float((e + 127) << 23); }
+
 // S^T for the 16 keys of this warp's block: rotated K fragments times Q^T.
 // Keys of rows g and g + 8 are rotated by the angles of positions pa and pb
-// (by minus those angles when sgn = -1).
-template <int D>
+// (by minus those angles when sgn = -1).  SCALED: each key row is first scaled
+// by its own power of two and ka / kc receive the inverse scales of rows
+// g / g + 8; otherwise the keys are rounded as they are and ka = kc = 1.
+template <int D, bool SCALED>
 __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int kw, int lane, uint32_t pa, uint32_t pb,
-                                             float sgn, const uint2* sturns, const uint32_t (&qb)[D / 16][2])
+                                             float sgn, const uint2* sturns, const uint32_t (&qb)[D / 16][2],
+                                             float& ka, float& kc)
 {
     const int t = lane & 3;
     c[0] = c[1] = c[2] = c[3] = 0.f;
     // ldmatrix.x4 rows: lanes 0-7 keys 0-7 / chunk lo, 8-15 keys 8-15 / lo, 16-23 keys 0-7 / hi, 24-31 keys 8-15 / hi
     const int lkey = kw + (lane & 7) + ((lane >> 3) & 1) * 8, lhalf = lane >> 4;
+    uint32_t lo[D / 32][4], hi[D / 32][4];
 #pragma unroll
     for (int kb = 0; kb < D / 32; ++kb) {
-        uint32_t lo[4], hi[4];
-        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + lhalf), lo);
-        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + D / 16 + lhalf), hi);
+        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + lhalf), lo[kb]);
+        ldsm_x4(dec_sw(ktile, lkey, 2 * kb + D / 16 + lhalf), hi[kb]);
+    }
+    float la = 1.f, lc = 1.f;
+    ka = kc = 1.f;
+    if (SCALED) {
+    // largest |k| of rows g (fragments 0, 2) and g + 8 (fragments 1, 3); the four
+    // threads t = 0..3 of a row hold its d values between them
+    uint32_t aa = 0u, ac = 0u;
+#pragma unroll
+    for (int kb = 0; kb < D / 32; ++kb) {
+        aa = absmax_bf16x2_dec(aa, absmax_bf16x2_dec(absmax_bf16x2_dec(lo[kb][0], lo[kb][2]),
+                                                     absmax_bf16x2_dec(hi[kb][0], hi[kb][2])));
+        ac = absmax_bf16x2_dec(ac, absmax_bf16x2_dec(absmax_bf16x2_dec(lo[kb][1], lo[kb][3]),
+                                                     absmax_bf16x2_dec(hi[kb][1], hi[kb][3])));
+    }
+    uint32_t ma = max(aa & 0x7fffu, (aa >> 16) & 0x7fffu), mc = max(ac & 0x7fffu, (ac >> 16) & 0x7fffu);
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+    mc = max(mc, __shfl_xor_sync(0xffffffffu, mc, 1));
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+    mc = max(mc, __shfl_xor_sync(0xffffffffu, mc, 2));
+    const int ea = range_exp_bf16(ma), ec = range_exp_bf16(mc);
+    la = pow2i_dec(ea);
+    lc = pow2i_dec(ec);
+    ka = pow2i_dec(-ea);
+    kc = pow2i_dec(-ec);
+    }
+#pragma unroll
+    for (int kb = 0; kb < D / 32; ++kb) {
         const int m0 = 16 * kb + 2 * t;
         // lo[0]: key g, dims m0,m0+1; lo[1]: key g+8; lo[2]: key g, dims m0+8,m0+9; lo[3]: key g+8
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const uint32_t pos = (r & 1) ? pb : pa;
+            const float lam = (r & 1) ? lc : la;
             const int m = m0 + ((r >> 1) ? 8 : 0);
             const uint2 w0 = sturns[m], w1 = sturns[m + 1];
             float c0, s0, c1, s1;
             rope_cs_fast(pos, w0.x, w0.y, c0, s0);
             rope_cs_fast(pos, w1.x, w1.y, c1, s1);
-            s0 *= sgn;
-            s1 *= sgn;
-            const float x0 = bf16_lo(lo[r]), x1 = bf16_hi(lo[r]);
-            const float y0 = bf16_lo(hi[r]), y1 = bf16_hi(hi[r]);
-            lo[r] = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
-            hi[r] = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
+            if (SCALED) {
+                c0 *= lam;
+                c1 *= lam;
+            }
+            s0 *= SCALED ? sgn * lam : sgn;
+            s1 *= SCALED ? sgn * lam : sgn;
+            const float x0 = bf16_lo(lo[kb][r]), x1 = bf16_hi(lo[kb][r]);
+            const float y0 = bf16_lo(hi[kb][r]), y1 = bf16_hi(hi[kb][r]);
+            lo[kb][r] = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+            hi[kb][r] = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
         }
-        mma_f16(c, lo, qb[kb][0], qb[kb][1]);
-        mma_f16(c, hi, qb[kb + D / 32][0], qb[kb + D / 32][1]);
+        mma_f16(c, lo[kb], qb[kb][0], qb[kb][1]);
+        mma_f16(c, hi[kb], qb[kb + D / 32][0], qb[kb + D / 32][1]);
     }
 }
 
@@ -502,6 +565,7 @@ __global__ void __launch_bounds__(TC_NT, 2)
     unsigned char* ring = smem;
     float* sq = reinterpret_cast<float*>(smem + C::SQ);           // [2][HPB][D]
     uint2* sturns = reinterpret_cast<uint2*>(smem + C::TURNS);    // (hi, lo) per frequency
+    int* qexp = reinterpret_cast<int*>(smem + C::QEXP);            // [HPB] query exponents
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BARS);
     uint64_t* empty = full + TC_STAGES;
     int* flag = reinterpret_cast<int*>(empty + TC_STAGES);
@@ -542,6 +606,41 @@ __global__ void __launch_bounds__(TC_NT, 2)
         }
     }
     __syncthreads();
+    // Query scales: a head whose rotated query (both rotations, base-2 logit
+    // units) has its largest |x| in [2^-3, 2^14) is used as it is (exponent 0);
+    // any other head is scaled to bring it into [2^13, 2^14).  Any scaled head,
+    // or an L1 norm above 2^14 (where fp16-subnormal keys could err by more than
+    // 2^-11 in a logit), sets qexp[8]: every key block of this CTA then takes the
+    // scaled path.  Warp w takes heads w, w + 5, ...
+    if (tid == 0) qexp[8] = 0;
+    __syncthreads();
+    for (int hh = warp; hh < HPB; hh += TC_NT / 32) {
+        float mx = 0.f, l1e = 0.f, l1r = 0.f;
+        for (int e = lane; e < D; e += 32) {
+            const float xe = fabsf(sq[(0 * HPB + hh) * D + e]), xr = fabsf(sq[(1 * HPB + hh) * D + e]);
+            mx = fmaxf(mx, fmaxf(xe, xr));
+            l1e += xe;
+            l1r += xr;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            l1e += __shfl_xor_sync(0xffffffffu, l1e, o);
+            l1r += __shfl_xor_sync(0xffffffffu, l1r, o);
+        }
+        // non-negative floats order like their bit patterns
+        const uint32_t bits = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+        if (lane == 0) {
+            int e = 0;
+            const float mxh = __uint_as_float(bits);
+            if (bits != 0u && bits < 0x7f800000u && !(mxh >= 0.125f && mxh < 16384.f)) {
+                const int biased = (int)(bits >> 23);
+                e = min(100, max(-100, 13 - ((biased == 0 ? 1 : biased) - 127)));
+            }
+            qexp[hh] = e;
+            if (e != 0 || !(fmaxf(l1e, l1r) <= 16384.f)) atomicOr(&qexp[8], 1);
+        }
+    }
+    __syncthreads();
 
     const int zkv = b * p.Hkv + kvh;
     float* mo = reinterpret_cast<float*>(ring);  // reused after the ring drains: [HPB][TC_NCW][D + 2]
@@ -551,12 +650,15 @@ __global__ void __launch_bounds__(TC_NT, 2)
             int issued = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % TC_STAGES;
-                if (c >= TC_STAGES && !mbar_wait(&empty[st], ((c / TC_STAGES) - 1) & 1)) {
+                if (c >= TC_STAGES && !mbar_wait(&empty[st], ((c / TC_STAGES) - 1) & 1, dl.wait_cycles)) {
                     record_error(dl.dev_error, 0x111);
                     break;
                 }
                 const int j0 = j_begin + c * TC_KROWS;
                 unsigned char* dst = ring + st * C::STAGE;
+                // (test hook: the first stage is never loaded, so the consumers'
+                // bounded waits on it expire)
+                if (c == 0 && dl.inject == kInjectDecodeCopy) continue;
                 mbar_arrive_expect_tx(&full[st], C::STAGE);
 #pragma unroll
                 for (int a = 0; a < C::ATOMS; ++a) {
@@ -566,7 +668,7 @@ __global__ void __launch_bounds__(TC_NT, 2)
                 issued = c + 1;
             }
             for (int c = max(0, issued - TC_STAGES); c < issued; ++c)
-                if (!mbar_wait(&full[c % TC_STAGES], (c / TC_STAGES) & 1)) record_error(dl.dev_error, 0x112);
+                if (!mbar_wait(&full[c % TC_STAGES], (c / TC_STAGES) & 1, dl.wait_cycles)) record_error(dl.dev_error, 0x112);
         }
         __syncthreads();
     } else {
@@ -574,16 +676,21 @@ __global__ void __launch_bounds__(TC_NT, 2)
         const int g = lane >> 2, t = lane & 3;
         // Q^T fragments (fp16): b0 = (Q[g][16kb+2t], Q[g][16kb+2t+1]), b1 = dims + 8; heads >= HPB are 0
         uint32_t qb_ex[D / 16][2], qb_rm[D / 16][2];
+        const float lq = g < HPB ? pow2i_dec(qexp[g]) : 1.f;
+        const bool always_scaled = qexp[8] != 0;
+        // inverse query scales of this thread's logit columns (heads 2t, 2t + 1)
+        const float cq0 = 2 * t < HPB ? pow2i_dec(-qexp[2 * t]) : 1.f;
+        const float cq1 = 2 * t + 1 < HPB ? pow2i_dec(-qexp[2 * t + 1]) : 1.f;
 #pragma unroll
         for (int kb = 0; kb < D / 16; ++kb) {
             const int m = 16 * kb + 2 * t;
             if (g < HPB) {
                 const float* qe = sq + (0 * HPB + g) * D;
                 const float* qr = sq + (1 * HPB + g) * D;
-                qb_ex[kb][0] = pack_f16x2(qe[m], qe[m + 1]);
-                qb_ex[kb][1] = pack_f16x2(qe[m + 8], qe[m + 9]);
-                qb_rm[kb][0] = pack_f16x2(qr[m], qr[m + 1]);
-                qb_rm[kb][1] = pack_f16x2(qr[m + 8], qr[m + 9]);
+                qb_ex[kb][0] = pack_f16x2(qe[m] * lq, qe[m + 1] * lq);
+                qb_ex[kb][1] = pack_f16x2(qe[m + 8] * lq, qe[m + 9] * lq);
+                qb_rm[kb][0] = pack_f16x2(qr[m] * lq, qr[m + 1] * lq);
+                qb_rm[kb][1] = pack_f16x2(qr[m + 8] * lq, qr[m + 9] * lq);
             } else {
                 qb_ex[kb][0] = qb_ex[kb][1] = qb_rm[kb][0] = qb_rm[kb][1] = 0u;
             }
@@ -596,7 +703,7 @@ __global__ void __launch_bounds__(TC_NT, 2)
         const int kw = warp * 16;  // this warp's keys within a stage
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % TC_STAGES;
-            if (!mbar_wait(&full[st], (c / TC_STAGES) & 1)) {
+            if (!mbar_wait(&full[st], (c / TC_STAGES) & 1, dl.wait_cycles)) {
                 record_error(dl.dev_error, 0x113);
                 break;
             }
@@ -609,17 +716,48 @@ __global__ void __launch_bounds__(TC_NT, 2)
             const uint32_t fa = div_g((uint32_t)ja, dl), fc = div_g((uint32_t)jc, dl);
             const uint32_t ra = p.rope_cache ? (uint32_t)ja - fa : fa, rc = p.rope_cache ? (uint32_t)jc - fc : fc;
             const float rsgn = p.rope_cache ? -1.f : 1.f;
+            // Keys are rounded to fp16 as they are unless that could lose the
+            // logits: an element beyond fp16's range (seen as a non-finite
+            // logit, as it always is) or a query for which the CTA takes the
+            // scaled path throughout.  Then each key row is scaled by its own
+            // power of two and the logits by the inverse key and query scales.
             float sc[4];
-            if (jb >= j_exact) {
-                block_logits<D>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex);
-            } else if (jb + 15 < j_exact) {
-                block_logits<D>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm);
-            } else {
-                float se[4];
-                block_logits<D>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm);
-                block_logits<D>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex);
-                if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
-                if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
+            bool scaled = always_scaled;
+            if (!scaled) {
+                float ka, kc;
+                if (jb >= j_exact) {
+                    block_logits<D, false>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                } else if (jb + 15 < j_exact) {
+                    block_logits<D, false>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                } else {
+                    float se[4];
+                    block_logits<D, false>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                    block_logits<D, false>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
+                    if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
+                }
+                scaled = __any_sync(0xffffffffu, !(fabsf(sc[0]) < INFINITY && fabsf(sc[1]) < INFINITY &&
+                                                   fabsf(sc[2]) < INFINITY && fabsf(sc[3]) < INFINITY));
+            }
+            if (scaled) {
+                float ka, kc;
+                if (jb >= j_exact) {
+                    block_logits<D, true>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                } else if (jb + 15 < j_exact) {
+                    block_logits<D, true>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                } else {
+                    float se[4];
+                    block_logits<D, true>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                    block_logits<D, true>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
+                    if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
+                }
+                // undo the operand scales: sc[0], sc[1] are key g with heads 2t,
+                // 2t + 1, sc[2], sc[3] key g + 8
+                sc[0] = sc[0] * ka * cq0;
+                sc[1] = sc[1] * ka * cq1;
+                sc[2] = sc[2] * kc * cq0;
+                sc[3] = sc[3] * kc * cq1;
             }
             if (ja >= j_end) sc[0] = sc[1] = -INFINITY;
             if (jc >= j_end) sc[2] = sc[3] = -INFINITY;
@@ -875,6 +1013,8 @@ cudaError_t launch_decode(const DecodeProblem& p, jetlong_dtype dt, cudaStream_t
     dl.partials = reinterpret_cast<float*>(p.workspace);
     dl.tickets = reinterpret_cast<unsigned int*>(reinterpret_cast<unsigned char*>(p.workspace) + part);
     dl.dev_error = p.dev_error;
+    dl.wait_cycles = p.wait_cycles > 0 ? p.wait_cycles : kDecodeWaitCycles;
+    dl.inject = p.inject;
     cudaError_t e = p.d == 64 ? dispatch<64>(p, dt, dl, s, false) : dispatch<128>(p, dt, dl, s, false);
     if (e == cudaSuccess) *nlaunch += 1;
     return e;
@@ -943,6 +1083,8 @@ cudaError_t launch_decode_noalloc(const DecodeProblem& p, jetlong_dtype dt, cuda
     dl.partials = reinterpret_cast<float*>(scratch);
     dl.tickets = reinterpret_cast<unsigned int*>(scratch + part);
     dl.dev_error = p.dev_error;
+    dl.wait_cycles = p.wait_cycles > 0 ? p.wait_cycles : kDecodeWaitCycles;
+    dl.inject = p.inject;
     e = p.d == 64 ? dispatch<64>(p, dt, dl, s, false) : dispatch<128>(p, dt, dl, s, false);
     if (e == cudaSuccess) *nlaunch += 1;
     return e;

@@ -21,6 +21,26 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};
+// Per-call largest |q|, |k| of bf16 prefills (written by the range scan, read
+// by the prefill kernel that follows it on the same stream).  Each call takes
+// the next of kRangeSlots pairs in turn, so calls in flight on different
+// streams use different words unless more than kRangeSlots prefill launches
+// are queued on the device at once.
+constexpr int kRangeSlots = 16384;
+__device__ uint32_t g_range_slots[2 * kRangeSlots];
+std::atomic<uint64_t> g_range_next{0};
+// one-shot failure-detection test hook of this host thread (jetlong_debug_inject_timeout)
+thread_local int g_inject_site = 0;
+thread_local long long g_inject_cycles = 0;
+
+// Takes the armed test hook, if any, for the attention launch being prepared.
+void take_injection(int* site, long long* cycles)
+{
+    *site = g_inject_site;
+    *cycles = g_inject_site ? g_inject_cycles : 0;
+    g_inject_site = 0;
+    g_inject_cycles = 0;
+}
 __device__ int g_dev_error;  // set by kernels whose bounded waits expire
 
 int fail(int code, const char* fmt, ...)
@@ -55,6 +75,28 @@ int* dev_error_word(cudaError_t* err)
         cache[dev] = static_cast<int*>(p);
     }
     return cache[dev];
+}
+
+// Device address of the next range slot pair (looked up once per device).
+uint32_t* next_range_slot(cudaError_t* err)
+{
+    static std::mutex mu;
+    static uint32_t* base[64] = {nullptr};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    uint32_t* b;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!base[dev]) {
+            void* ptr = nullptr;
+            *err = cudaGetSymbolAddress(&ptr, g_range_slots);
+            if (*err != cudaSuccess) return nullptr;
+            base[dev] = static_cast<uint32_t*>(ptr);
+        }
+        b = base[dev];
+    }
+    return b + 2 * (g_range_next.fetch_add(1) % kRangeSlots);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -162,6 +204,18 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.dev_error = derr;
     int n = 0;
+    if (dtype == JETLONG_BF16) {
+        // largest |q| and |k| of the rows this call uses, for the power-of-two
+        // operand scales of the fp16 Q K^T (see range_scan.cu)
+        uint32_t* slot = next_range_slot(&e);
+        if (!slot) return fail(JETLONG_ERR_CUDA, "range slots: %s", cudaGetErrorString(e));
+        e = jl::launch_range_scan(q, C, Cst, B * Hq, k, L, Lcap, B * Hkv, d, slot, (cudaStream_t)stream, &n);
+        g_launches += n;
+        n = 0;
+        if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "range scan launch: %s", cudaGetErrorString(e));
+        p.range = slot;
+    }
+    take_injection(&p.inject, &p.wait_cycles);
     // bf16: tensor-core kernel; fp32: CUDA-core fp32 kernel (TF32 would miss fp32 accuracy)
     e = dtype == JETLONG_BF16 ? jl::launch_prefill_tc(p, (cudaStream_t)stream, &n)
                               : jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
@@ -353,6 +407,26 @@ int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void*
     // the caller's stream continues once the last rows are back on the host
     if (e == cudaSuccess && st == JETLONG_OK && (e = cudaEventRecord(ev[2 * nch + 1], d2h)) == cudaSuccess)
         e = cudaStreamWaitEvent(cs, ev[2 * nch + 1], 0);
+    if (e != cudaSuccess || st != JETLONG_OK) {
+        // a failure part-way: copies may still be queued on the library's copy
+        // streams; make the caller's stream (and so anything it later frees or
+        // reuses) wait for them, or wait here if even that cannot be arranged
+        const std::string msg = g_last_error;
+        cudaEvent_t tail[2] = {nullptr, nullptr};
+        bool joined = true;
+        for (int i = 0; i < 2; ++i) {
+            cudaStream_t src = i == 0 ? h2d : d2h;
+            joined = joined && cudaEventCreateWithFlags(&tail[i], cudaEventDisableTiming) == cudaSuccess &&
+                     cudaEventRecord(tail[i], src) == cudaSuccess && cudaStreamWaitEvent(cs, tail[i], 0) == cudaSuccess;
+        }
+        if (!joined) {
+            cudaStreamSynchronize(h2d);
+            cudaStreamSynchronize(d2h);
+        }
+        for (auto& x : tail)
+            if (x) cudaEventDestroy(x);
+        g_last_error = msg;
+    }
     release();
     if (st != JETLONG_OK) return st;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "streamed prefill: %s", cudaGetErrorString(e));
@@ -401,6 +475,7 @@ static int decode_entry(const void* q, const void* kcache, const void* vcache, v
     p.workspace = workspace;
     p.workspace_bytes = workspace_bytes;
     p.dev_error = derr;
+    take_injection(&p.inject, &p.wait_cycles);
     int n = 0;
     e = jl::launch_decode(p, dtype, (cudaStream_t)stream, &n);
     g_launches += n;
@@ -452,6 +527,7 @@ int jetlong_decode_noalloc(const void* q, const void* kcache, const void* vcache
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.dev_error = derr;
+    take_injection(&p.inject, &p.wait_cycles);
     int n = 0;
     size_t need = 0;
     e = jl::launch_decode_noalloc(p, dtype, (cudaStream_t)stream, &n, &need);
@@ -474,6 +550,17 @@ int jetlong_selftest_wait_timeout(void* stream)
     e = jl::launch_wait_selftest(derr, 2000000ll, (cudaStream_t)stream, &n);  // ~1 ms
     g_launches += n;
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int jetlong_debug_inject_timeout(int site, long long wait_cycles)
+{
+    if (site < JETLONG_INJECT_NONE || site > JETLONG_INJECT_DECODE_COPY)
+        return fail(JETLONG_ERR_INVALID_ARG, "unknown injection site %d", site);
+    if (site != JETLONG_INJECT_NONE && (wait_cycles < 10000 || wait_cycles > 4000000000ll))
+        return fail(JETLONG_ERR_INVALID_ARG, "wait_cycles must be in [1e4, 4e9] (got %lld)", wait_cycles);
+    g_inject_site = site;
+    g_inject_cycles = wait_cycles;
     return ok();
 }
 

@@ -105,6 +105,11 @@ struct PrefillProblem {
     float scale_log2;  // scale * log2(e): logits kept in base-2 units
     RopeTurns turns;
     int* dev_error;    // device error word (bounded waits)
+    long long wait_cycles;  // limit of every bounded wait of the attention roles
+    int inject;             // failure-detection test hook (kInjectNone in normal calls)
+    // bf16: two words (largest |q|, largest |k| as bf16 magnitude bits) written
+    // by launch_range_scan on the same stream before the prefill kernel
+    const uint32_t* range;
 };
 
 struct DecodeProblem {
@@ -118,7 +123,21 @@ struct DecodeProblem {
     void* workspace;
     size_t workspace_bytes;
     int* dev_error;
+    long long wait_cycles;
+    int inject;
 };
+
+// Failure-detection test hook: the barrier arrival a launch withholds (the
+// values of jetlong_debug_inject_timeout's `site`).
+enum {
+    kInjectNone = 0,
+    kInjectPrefillKeyTile = JETLONG_INJECT_PREFILL_KEY_TILE,  // bf16 prefill: the first key tile is never released
+    kInjectDecodeCopy = JETLONG_INJECT_DECODE_COPY,           // bf16 decode: the first K/V stage is never loaded
+};
+// Normal limits: ~0.5 s for the prefill roles, ~2 s for the decode (every wait
+// is on work of the same CTA or CTA pair).
+constexpr long long kPrefillWaitCycles = 1000000000ll;
+constexpr long long kDecodeWaitCycles = 4000000000ll;
 
 // Returns cudaSuccess or the launch error; each adds its launches to *nlaunch.
 cudaError_t launch_prefill_simt(const PrefillProblem& p, jetlong_dtype dt, cudaStream_t s,
@@ -137,5 +156,10 @@ cudaError_t launch_ie_merge(const void* oa, const void* ob, const void* oc, cons
                             const float* lc, void* out, long long rows, int d, jetlong_dtype dt,
                             cudaStream_t s, int* nlaunch);
 cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStream_t s, int* nlaunch);
+// Largest magnitude of the used rows of q (planes of Cst rows, rows [0, C)) and
+// of k (planes of Lcap rows, rows [0, L)), bf16, as 15-bit magnitude bits into
+// range[0] and range[1] (zeroed first on the stream).
+cudaError_t launch_range_scan(const void* q, int C, int Cst, int q_planes, const void* k, int L, int Lcap,
+                              int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch);
 
 }  // namespace jl

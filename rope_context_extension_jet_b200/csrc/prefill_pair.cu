@@ -151,14 +151,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             for (int e = 0; e < NE; ++e) {
                 const int kb = tp.kb(e);
                 const int s = e % NS, u = e / NS;
-                if (e >= NS && !wait_or_abort<true>(&bars[P_KEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, 0x401)) break;
+                if (e >= NS && !wait_or_abort<true>(&bars[P_KEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x401)) break;
                 mbar_arrive_expect_tx(&bars[P_KFULL + s], S::KTILE);
 #pragma unroll
                 for (int a = 0; a < 2; ++a)
                     tma_load_3d(smem + S::K0 + s * S::KTILE + a * S::KATOM, &tmK, a * 64, kb * BN + (int)rank * KROWS,
                                 zkv, &bars[P_KFULL + s]);
                 k_issued = e + 1;
-                if (e >= NS && !wait_or_abort<true>(&bars[P_VEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, 0x402)) break;
+                if (e >= NS && !wait_or_abort<true>(&bars[P_VEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x402)) break;
                 mbar_arrive_expect_tx(&bars[P_VFULL + s], S::VTILE);
                 tma_load_3d(smem + S::V0 + s * S::VTILE, &tmV, (int)rank * 64, kb * BN, zkv, &bars[P_VFULL + s]);
                 v_issued = e + 1;
@@ -197,15 +197,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             // V half of tile pe landed in both CTAs and P_h of tile pe is in both TMEMs
             auto pv_ready = [&](int h, int pe) {
                 const int s = pe % NS, u = pe / NS;
-                return warp_wait<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, 0x411 + h) &&
-                       (h == 1 || (warp_wait(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x413) &&
-                                   warp_wait<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, 0x414)));
+                return warp_wait<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x411 + h) &&
+                       (h == 1 || (warp_wait(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x413) &&
+                                   warp_wait<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x414)));
             };
             // Issue order per tile e: P_0 V (tile e-1), Q_0 K^T (tile e), P_1 V
             // (tile e-1), Q_1 K^T (tile e).  S_h(e) overwrites P_h(e-1) in TMEM;
             // the P.V reading it was issued earlier by this warp and the tensor
             // pipe runs one issuer's MMAs in issue order.
-            bool ok = warp_wait<true>(&bars[P_QREADY0], 0, abort_flag, p.dev_error, 0x415);
+            bool ok = warp_wait<true>(&bars[P_QREADY0], 0, abort_flag, p.dev_error, p.wait_cycles, 0x415);
             tc_fence_after();
             for (int e = 0; e < NE && ok; ++e) {
                 const int s = e % NS, u = e / NS, pe = e - 1, ps = (e + NS - 1) % NS;
@@ -217,9 +217,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 if (e == nR && nR > 0) {
                     // Q of phase R is no longer read once every MMA so far completed
                     umma_commit_pair_both_elect(&bars[P_QFREE]);
-                    if (!warp_wait<true>(&bars[P_QREADY1], 0, abort_flag, p.dev_error, 0x416)) { ok = false; break; }
+                    if (!warp_wait<true>(&bars[P_QREADY1], 0, abort_flag, p.dev_error, p.wait_cycles, 0x416)) { ok = false; break; }
                 }
-                if (!warp_wait<true>(&bars[P_KREADY + s], u & 1, abort_flag, p.dev_error, 0x417)) { ok = false; break; }
+                if (!warp_wait<true>(&bars[P_KREADY + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x417)) { ok = false; break; }
                 tc_fence_after();
                 qk(0, s);
                 if (e > 0) {
@@ -251,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             // ---------------------------------------------------------- V relay (CTA 1)
             for (int e = 0; e < NE; ++e) {
                 const int s = e % NS, u = e / NS;
-                if (!wait_or_abort(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, 0x421)) break;
+                if (!wait_or_abort(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x421)) break;
                 mbar_arrive_cluster(lead(P_VPEER + s));
             }
         }
@@ -261,14 +261,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
+        // operand scales of this call (powers of two, see range_exp)
+        const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
         const uint32_t i0 = (uint32_t)(p.P + qb * BM);
-        bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, 0x431);
+        bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, p.wait_cycles, 0x431);
         if (ok) {
             for (int h = 0; h < 2; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                                             sts, lq);
                 else
-                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -279,24 +282,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const int s = e % NS, u = e / NS;
             if (e == nR && nR > 0) {
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
-                if (!warp_wait<true>(&bars[P_QFREE], 0, abort_flag, p.dev_error, 0x432)) { ok = false; break; }
+                if (!warp_wait<true>(&bars[P_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x432)) { ok = false; break; }
                 for (int h = 0; h < 2; ++h)
                     rotate_tile<D, BM, false>(smem + h * S::QTILE, t, p,
-                                              [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts);
+                                              [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(lead(P_QREADY1));
             }
-            if (!warp_wait(&bars[P_KFULL + s], u & 1, abort_flag, p.dev_error, 0x433)) { ok = false; break; }
+            if (!warp_wait(&bars[P_KFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x433)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
             unsigned char* kt = smem + S::K0 + s * S::KTILE;
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
+                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts, lk);
             else
-                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts);
+                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead(P_KREADY + s));
+            // (test hook: the first key tile is never released, so the MMA warp's
+            // bounded wait on it expires)
+            if (lane == 0 && !(p.inject == kInjectPrefillKeyTile && e == 0)) mbar_arrive_cluster(lead(P_KREADY + s));
         }
     } else {
         regs_inc<192>();

@@ -143,14 +143,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int e = 0; e < NE; ++e) {
                 const int kb = tp.kb(e);
                 const int sk = e % NSK, uk = e / NSK;
-                if (e >= NSK && !wait_or_abort(&bars[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, p.dev_error, 0x301)) break;
+                if (e >= NSK && !wait_or_abort(&bars[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x301)) break;
                 mbar_arrive_expect_tx(&bars[B_KFULL + sk], S::TILE);
 #pragma unroll
                 for (int a = 0; a < S::ATOMS; ++a)
                     tma_load_3d(smem + S::K0 + sk * S::TILE + a * ATOM, &tmK, a * 64, kb * BN, zkv, &bars[B_KFULL + sk]);
                 k_issued = e + 1;
                 const int sv = e % NSV, uv = e / NSV;
-                if (e >= NSV && !wait_or_abort(&bars[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, p.dev_error, 0x302)) break;
+                if (e >= NSV && !wait_or_abort(&bars[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x302)) break;
                 mbar_arrive_expect_tx(&bars[B_VFULL + sv], S::TILE);
 #pragma unroll
                 for (int a = 0; a < S::ATOMS; ++a)
@@ -184,44 +184,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                  sdesc_sw128(vaddr + k * 2048, ATOM, 1024), IDESC_PV, (!first || k > 0) ? 1u : 0u);
                 umma_commit(&bars[B_PVDONE + h]);
             };
-            bool ok = wait_or_abort(&bars[B_QREADY0], 0, abort_flag, p.dev_error, 0x311);
+            bool ok = wait_or_abort(&bars[B_QREADY0], 0, abort_flag, p.dev_error, p.wait_cycles, 0x311);
             tc_fence_after();
             for (int e = 0; e < NE && ok; ++e) {
                 const int sk = e % NSK, uk = e / NSK, sv = e % NSV, uv = e / NSV;
                 if (e == nR && nR > 0) {
                     // Q of phase R is no longer read once every MMA so far completed
                     umma_commit(&bars[B_QFREE]);
-                    if (!wait_or_abort(&bars[B_QREADY1], 0, abort_flag, p.dev_error, 0x312)) { ok = false; break; }
+                    if (!wait_or_abort(&bars[B_QREADY1], 0, abort_flag, p.dev_error, p.wait_cycles, 0x312)) { ok = false; break; }
                 }
-                if (!wait_or_abort(&bars[B_KREADY + sk], uk & 1, abort_flag, p.dev_error, 0x313)) { ok = false; break; }
-                if (e > 0 && !wait_or_abort(&bars[B_PVDONE + 0], (e - 1) & 1, abort_flag, p.dev_error, 0x314)) { ok = false; break; }
+                if (!wait_or_abort(&bars[B_KREADY + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x313)) { ok = false; break; }
+                if (e > 0 && !wait_or_abort(&bars[B_PVDONE + 0], (e - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x314)) { ok = false; break; }
                 tc_fence_after();
                 qk(0, sk);
                 if (NH == 2) {
                     if (e > 0) {
                         // head 1's P.V of the previous tile runs while head 0's softmax works
                         const int pe = e - 1, psv = pe % NSV, puv = pe / NSV;
-                        if (!wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, 0x315)) { ok = false; break; }
-                        if (!wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, 0x316)) { ok = false; break; }
+                        if (!wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x315)) { ok = false; break; }
+                        if (!wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x316)) { ok = false; break; }
                         tc_fence_after();
                         pv(1, psv, pe == 0);
                         umma_commit(&bars[B_VEMPTY + psv]);
-                        if (!wait_or_abort(&bars[B_PVDONE + 1], pe & 1, abort_flag, p.dev_error, 0x317)) { ok = false; break; }
+                        if (!wait_or_abort(&bars[B_PVDONE + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x317)) { ok = false; break; }
                         tc_fence_after();
                     }
                     qk(1, sk);
                 }
                 umma_commit(&bars[B_KEMPTY + sk]);
-                if (!wait_or_abort(&bars[B_PFULL + 0], e & 1, abort_flag, p.dev_error, 0x318)) { ok = false; break; }
-                if (!wait_or_abort(&bars[B_VFULL + sv], uv & 1, abort_flag, p.dev_error, 0x319)) { ok = false; break; }
+                if (!wait_or_abort(&bars[B_PFULL + 0], e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x318)) { ok = false; break; }
+                if (!wait_or_abort(&bars[B_VFULL + sv], uv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x319)) { ok = false; break; }
                 tc_fence_after();
                 pv(0, sv, e == 0);
                 if (NH == 1) umma_commit(&bars[B_VEMPTY + sv]);
             }
             if (ok && NH == 2 && NE > 0) {
                 const int pe = NE - 1, psv = pe % NSV, puv = pe / NSV;
-                if (wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, 0x31a) &&
-                    wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, 0x31b)) {
+                if (wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31a) &&
+                    wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31b)) {
                     tc_fence_after();
                     pv(1, psv, pe == 0);
                     umma_commit(&bars[B_VEMPTY + psv]);
@@ -237,14 +237,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int t = tid - 128;
         float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
+        // operand scales of this call (powers of two, see range_exp)
+        const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
         const uint32_t i0 = (uint32_t)(p.P + qb * BM);
-        bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, 0x321);
+        bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, p.wait_cycles, 0x321);
         if (ok) {
             for (int h = 0; h < NH; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                                             sts, lq);
                 else
-                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts);
+                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -255,23 +258,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int sk = e % NSK, uk = e / NSK;
             if (e == nR && nR > 0) {
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
-                if (!warp_wait(&bars[B_QFREE], 0, abort_flag, p.dev_error, 0x322)) { ok = false; break; }
+                if (!warp_wait(&bars[B_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x322)) { ok = false; break; }
                 for (int h = 0; h < NH; ++h)
                     rotate_tile<D, BM, false>(smem + h * S::TILE, t, p,
-                                          [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts);
+                                          [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_QREADY1]);
             }
-            if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, 0x323)) { ok = false; break; }
+            if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x323)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN);
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts);
+                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc,
+                                         sts, lk);
             else
-                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts);
+                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_KREADY + sk]);
+            // (test hook: the first key tile is never released, so the MMA
+            // thread's bounded wait on it expires)
+            if (lane == 0 && !(p.inject == kInjectPrefillKeyTile && e == 0)) mbar_arrive(&bars[B_KREADY + sk]);
         }
     } else {
         regs_inc<184>();
@@ -374,6 +380,9 @@ TcParams make_params(const PrefillProblem& pp)
     p.lse = pp.lse;
     p.window_rot = pp.window_rot;
     p.dev_error = pp.dev_error;
+    p.wait_cycles = pp.wait_cycles > 0 ? pp.wait_cycles : kPrefillWaitCycles;
+    p.inject = pp.inject;
+    p.range = pp.range;
     return p;
 }
 

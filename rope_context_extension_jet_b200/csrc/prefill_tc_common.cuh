@@ -23,7 +23,6 @@ namespace tc {
 
 constexpr int BM = 128, BN = 128;
 constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
-constexpr long long kTcWaitCycles = 1000000000ll;  // ~0.5 s: every wait here is on work of this CTA (pair)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
 enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
@@ -40,7 +39,43 @@ struct TcParams {
     float* lse;      // optional
     int window_rot;  // -1 routed; 0 / 1: pairs i - j < w0 only, exact / aliased rotation
     int* dev_error;
+    long long wait_cycles;  // limit of every bounded wait
+    int inject;             // kInjectNone, or the arrival this launch withholds (test hook)
+    // largest |q| and |k| of this call as bf16 magnitude bits, written by the
+    // range scan launched just before on the same stream
+    const uint32_t* range;
 };
+
+// ------------------------------------------------------------ operand range
+// The Q K^T operands are rounded to fp16 (an 11-bit significand: the inputs'
+// 8-bit bf16 significand would cost the logits too much precision), whose range
+// ends at 65504 while bf16 inputs reach 3.4e38.  So the rotated queries and keys
+// are scaled by powers of two 2^e_q and 2^e_k that bring the call's largest
+// |q| and |k| into [2^13, 2^14): a rotated value is at most sqrt(2) times the
+// largest input of its pair, so every operand stays below 2^14.5, and inputs
+// down to 2^27 below the largest keep fp16's full relative precision (smaller
+// ones become subnormal or zero; their part of a logit is then below 2^-38 of
+// the largest terms).  A power of two is exact both ways, so the softmax, which
+// multiplies S by scale * log2(e) * 2^-(e_q + e_k), sees the logits of the
+// unscaled operands; for inputs already in range the result is bit-identical.
+// Exponents are clamped to [-100, 100].
+__device__ __forceinline__ int range_exp(uint32_t mag)
+{
+    if (mag == 0u || mag >= 0x7f80u) return 0;  // all zero, or non-finite: nothing to rescale
+    const int biased = (int)(mag >> 7);
+    const int ilogb = (biased == 0 ? 1 : biased) - 127;  // subnormals: at most 2^-126
+    return min(100, max(-100, 13 - ilogb));
+}
+
+// 2^e as fp32 for e in [-126, 127].
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+__device__ __forceinline__ uint32_t ld_range(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ uint32_t div_g(uint32_t n, const TcParams& p)
 {
@@ -97,13 +132,13 @@ __device__ __forceinline__ bool bar_try_wait(uint64_t* bar, uint32_t parity)
 // or MMA commits from the other CTA of a pair).
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int* dev_error, int code)
+                                              int* dev_error, long long limit, int code)
 {
     if (bar_try_wait<CLUSTER>(bar, parity)) return true;
     const long long t0 = clock64();
     while (!bar_try_wait<CLUSTER>(bar, parity)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kTcWaitCycles) {
+        if (clock64() - t0 > limit) {
             record_error(dev_error, code);
             *abort_flag = 1;
             return false;
@@ -115,9 +150,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // Warp-collective form: every lane polls, and the warp proceeds only if all did.
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* dev_error, int code)
+                                          int* dev_error, long long limit, int code)
 {
-    const bool ok = wait_or_abort<CLUSTER>(bar, parity, abort_flag, dev_error, code);
+    const bool ok = wait_or_abort<CLUSTER>(bar, parity, abort_flag, dev_error, limit, code);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -133,7 +168,7 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int ch)
 __device__ __forceinline__ float f16_lo(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu))); }
 __device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
 
-// RoPE of a ROWS-row tile in place (pairs (m, m + d/2)), output fp16.  Thread t
+// RoPE of a ROWS-row tile in place (pairs (m, m + d/2)), times lam, output fp16.  Thread t
 // of the 128 rotation threads owns 8 frequencies (chunk c) of RPT consecutive
 // rows.  pos(row) must step by 0 or 1 between consecutive rows (true for j,
 // floor(j/G) and i - floor(i/G)); the angles of the first row come from the
@@ -141,15 +176,21 @@ __device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__usho
 // rotation R(theta_m) (any other step is recomputed exactly).
 template <int D, int ROWS, bool IN_BF16, class PosFn>
 __device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const TcParams& p, PosFn pos,
-                                            const float (&stc)[8], const float (&sts)[8])
+                                            const float (&stc)[8], const float (&sts)[8], float lam)
 {
     constexpr int H = D / 2, CH = H / 8, RPT = ROWS * CH / 128;  // 128 threads = CH chunks x (ROWS / RPT) row groups
     static_assert(RPT >= 1 && ROWS * CH == 128 * RPT, "rotation thread mapping");
     const int c = t % CH, row0 = (t / CH) * RPT;
+    // (cs, sn) carry the operand scale lam: the step rotation is linear, so
+    // every row it produces keeps it
     float cs[8], sn[8];
     uint32_t prev = pos(row0);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) rope_cs_fast(prev, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+    for (int u = 0; u < 8; ++u) {
+        rope_cs_fast(prev, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+        cs[u] *= lam;
+        sn[u] *= lam;
+    }
 #pragma unroll 2
     for (int s = 0; s < RPT; ++s) {
         const int r = row0 + s;
@@ -164,7 +205,11 @@ __device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const Tc
                 }
             } else if (cur != prev) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) rope_cs_fast(cur, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+                for (int u = 0; u < 8; ++u) {
+                    rope_cs_fast(cur, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
+                    cs[u] *= lam;
+                    sn[u] *= lam;
+                }
             }
             prev = cur;
         }
@@ -216,14 +261,18 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
     const int i_lo = p.P + qb * BM;
     const int i = i_lo + r;
     const int NE = tp.count();
-    const float sl2 = p.scale_log2;
+    // scale * log2(e), times 2^-(e_q + e_k) to undo the operand scales; kept in
+    // fp32's normal range, so a masked -inf column never meets a zero or
+    // infinite factor (logits that small or large are outside fp32 anyway)
+    const float sl2 = fminf(fmaxf(p.scale_log2 * pow2i(-range_exp(ld_range(p.range))) *
+                                  pow2i(-range_exp(ld_range(p.range + 1))), 1.17549435e-38f), 3.40282347e38f);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int e = 0; e < NE; ++e) {
         const int kb = tp.kb(e);
         const bool phase_r = e < tp.nR;
         const int cls = tile_class(i_lo, kb, L, p.w0);
-        if (!warp_wait<CLUSTER>(sfull, e & 1, abort_flag, p.dev_error, 0x331)) { ok = false; break; }
+        if (!warp_wait<CLUSTER>(sfull, e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x331)) { ok = false; break; }
         tc_fence_after();
         float x[BN];
         {
@@ -292,7 +341,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
         // MMA of that thread.  So P may overwrite its columns now; the rare O
         // rescale still checks pvdone explicitly.
         if (e > 0 && __any_sync(0xffffffffu, resc)) {
-            if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, 0x332)) { ok = false; break; }
+            if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x332)) { ok = false; break; }
             tc_fence_after();
             {
 #pragma unroll
@@ -319,7 +368,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
         if (lane == 0) arrive_p();
     }
     // epilogue: O / l -> bf16 -> out
-    if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, 0x333)) {
+    if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x333)) {
         tc_fence_after();
         const float inv = 1.f / l;
         const size_t row = ((size_t)b * p.Hq + head) * (size_t)p.Cst + (size_t)(i - p.P);

@@ -221,3 +221,14 @@ def test_decode_noalloc_rejects_bad_arguments_on_host(lib, kw, status):
     assert _noalloc(lib, **kw) == status
     assert jl.launch_count() == before
     assert jl.last_error() != ""
+
+
+def test_injection_hook_arguments(lib):
+    # failure-detection test hook: unknown sites and out-of-range limits are refused
+    assert lib.jetlong_debug_inject_timeout(3, 2_000_000) == 1
+    assert lib.jetlong_debug_inject_timeout(-1, 2_000_000) == 1
+    assert lib.jetlong_debug_inject_timeout(1, 9_999) == 1
+    assert lib.jetlong_debug_inject_timeout(2, 4_000_000_001) == 1
+    assert "wait_cycles" in lib.jetlong_last_error().decode()
+    assert lib.jetlong_debug_inject_timeout(1, 2_000_000) == 0
+    assert lib.jetlong_debug_inject_timeout(0, 0) == 0  # disarmed again

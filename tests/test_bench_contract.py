@@ -100,3 +100,25 @@ def test_peak_clock_lookup_searches_nested_keys():
     d = {"hbm_gbs": 6548.5, "bf16": {"sustained": {"sm_mhz_median_sustained": 1335}, "burst_sm_mhz": 1900},
          "mem_clock_mhz_sustained": 3996}
     assert bench._find_mhz(d, "sustain") == 1335.0
+
+
+NCU_CSV = '''==PROF== Connected to process 4242
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","4242","python3","127.0.0.1","prefill_pair_kernel(CUtensorMap_st, CUtensorMap_st, CUtensorMap_st, jl::tc::TcParams)","1","7","(512, 1, 1)","(2048, 8, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","ns","156,000,000"
+"1","4242","python3","127.0.0.1","void jl::decode_tc_kernel<128, 4>(CUtensorMap_st, CUtensorMap_st, jl::DecodeProblem, jl::DecodeLaunch)","1","7","(160, 1, 1)","(4, 8, 8)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","ns","800000"
+"2","4242","python3","127.0.0.1","void jl::decode_tc_kernel<128, 4>(CUtensorMap_st, CUtensorMap_st, jl::DecodeProblem, jl::DecodeLaunch)","1","7","(160, 1, 1)","(4, 8, 8)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","ns","1200000"
+"2","4242","python3","127.0.0.1","void jl::decode_tc_kernel<128, 4>(CUtensorMap_st, CUtensorMap_st, jl::DecodeProblem, jl::DecodeLaunch)","1","7","(160, 1, 1)","(4, 8, 8)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","4,294,967,296"
+==PROF== Disconnected from process 4242
+'''
+
+
+def test_ncu_csv_parsing_and_launch_shares():
+    rows = bench.parse_ncu_csv(NCU_CSV)
+    assert len(rows) == 4
+    assert rows[0]["value"] == 156e6 and rows[3]["value"] == 4294967296.0
+    summ = bench.launch_summary(rows)
+    assert [s[0] for s in summ] == ["prefill_pair_kernel", "void jl::decode_tc_kernel<128, 4>"]
+    (k0, n0, t0, s0), (k1, n1, t1, s1) = summ
+    assert (n0, n1) == (1, 2)
+    assert t0 == pytest.approx(156.0) and t1 == pytest.approx(2.0)
+    assert s0 == pytest.approx(156.0 / 158.0) and s0 + s1 == pytest.approx(1.0)
