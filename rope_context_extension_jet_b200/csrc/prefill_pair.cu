@@ -176,22 +176,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             constexpr uint32_t IDESC_PV = idesc_bf16(2 * BM, D, 1);
             const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
             const uint32_t sbase = smem_u32(smem);
+            // (the step offsets inside umma_pair_qk_k128 / _pv_k128 are those of
+            // these tiles: Q atoms 16 KB apart, K-half atoms 8 KB apart, V slices 2 KB)
+            static_assert(ATOM == 1024 * 16 && S::KATOM == 512 * 16 && BN / 16 == 8 && D / 16 == 8,
+                          "tile layout of the grouped MMA issue");
             auto qk = [&](int h, int s) {
                 const uint32_t qaddr = sbase + h * S::QTILE, kaddr = sbase + S::K0 + s * S::KTILE;
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    umma_pair_ss_elect(tm + h * 128, sdesc_sw128(qaddr + (k >> 2) * ATOM + (k & 3) * 32, 16, 1024),
-                                       sdesc_sw128(kaddr + (k >> 2) * S::KATOM + (k & 3) * 32, 16, 1024), IDESC_QK,
-                                       k > 0 ? 1u : 0u);
+                umma_pair_qk_k128(tm + h * 128, sdesc_sw128(qaddr, 16, 1024), sdesc_sw128(kaddr, 16, 1024), IDESC_QK, 0u);
                 umma_commit_pair_both_elect(&bars[P_SFULL + h]);
             };
             auto pv = [&](int h, int s, bool first) {
                 const uint32_t vaddr = sbase + S::V0 + s * S::VTILE;
-#pragma unroll
-                for (int k = 0; k < BN / 16; ++k)
-                    umma_pair_ts_elect(tm + 256 + h * 128, tm + h * 128 + k * 8,
-                                       sdesc_sw128(vaddr + k * 2048, S::VTILE, 1024), IDESC_PV,
-                                       (!first || k > 0) ? 1u : 0u);
+                umma_pair_pv_k128(tm + 256 + h * 128, tm + h * 128, sdesc_sw128(vaddr, S::VTILE, 1024), IDESC_PV,
+                                  first ? 0u : 1u);
                 umma_commit_pair_both_elect(&bars[P_PVDONE + h]);
             };
             // V half of tile pe landed in both CTAs and P_h of tile pe is in both TMEMs

@@ -24,8 +24,9 @@
 //
 // Warp roles (512 threads, 4 warpgroups; registers rebalanced with setmaxnreg):
 //   warp 0        TMA producer (raw Q once; raw K and V per tile)
-//   warp 1        MMA issuer (one thread): S_h = Q_h K^T (fp16 operands) into
-//                 TMEM; O_h += P_h V with P_h read from TMEM (bf16)
+//   warp 1        MMA issuer (the whole warp; one elected lane issues each
+//                 group of MMAs): S_h = Q_h K^T (fp16 operands) into TMEM;
+//                 O_h += P_h V with P_h read from TMEM (bf16)
 //   warp 2        TMEM allocation / release
 //   warps 4-7     rotation: RoPE of Q and of every K tile in shared memory,
 //                 angles advanced row by row with a per-frequency rotation step
@@ -161,74 +162,76 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait(&bars[B_QFULL], 0);
             for (int ee = max(0, k_issued - NSK); ee < k_issued; ++ee) mbar_wait(&bars[B_KFULL + ee % NSK], (ee / NSK) & 1);
             for (int ee = max(0, v_issued - NSV); ee < v_issued; ++ee) mbar_wait(&bars[B_VFULL + ee % NSV], (ee / NSV) & 1);
-        } else if (warp == 1 && lane == 0) {
+        } else if (warp == 1) {
             // ---------------------------------------------------------- MMA issuer
+            // The whole warp runs the loop with warp-uniform values and waits; one
+            // elected lane issues each group of MMAs and each commit.
             constexpr uint32_t IDESC_QK = idesc_f16(BM, BN, 0);
             constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 1);
+            static_assert(ATOM == 1024 * 16 && BN / 16 == 8 && (D == 64 || D == 128),
+                          "tile layout of the grouped MMA issue");
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
             const uint32_t sbase = smem_u32(smem);
             auto qk = [&](int h, int sk) {
-                const uint32_t qaddr = sbase + h * S::TILE, kaddr = sbase + S::K0 + sk * S::TILE;
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t off = (k >> 2) * ATOM + (k & 3) * 32;
-                    umma_bf16_ss(tmem + h * 128, sdesc_sw128(qaddr + off, 16, 1024),
-                                 sdesc_sw128(kaddr + off, 16, 1024), IDESC_QK, k > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[B_SFULL + h]);
+                const uint64_t a = sdesc_sw128(sbase + h * S::TILE, 16, 1024);
+                const uint64_t bk = sdesc_sw128(sbase + S::K0 + sk * S::TILE, 16, 1024);
+                if (D == 128)
+                    umma_qk_k128(tm + h * 128, a, bk, IDESC_QK);
+                else
+                    umma_qk_k64(tm + h * 128, a, bk, IDESC_QK);
+                umma_commit_elect(&bars[B_SFULL + h]);
             };
             auto pv = [&](int h, int sv, bool first) {
-                const uint32_t vaddr = sbase + S::V0 + sv * S::TILE;
-#pragma unroll
-                for (int k = 0; k < BN / 16; ++k)
-                    umma_bf16_ts(tmem + 256 + h * 128, tmem + h * 128 + k * 8,
-                                 sdesc_sw128(vaddr + k * 2048, ATOM, 1024), IDESC_PV, (!first || k > 0) ? 1u : 0u);
-                umma_commit(&bars[B_PVDONE + h]);
+                umma_pv_k128(tm + 256 + h * 128, tm + h * 128, sdesc_sw128(sbase + S::V0 + sv * S::TILE, ATOM, 1024),
+                             IDESC_PV, first ? 0u : 1u);
+                umma_commit_elect(&bars[B_PVDONE + h]);
             };
-            bool ok = wait_or_abort(&bars[B_QREADY0], 0, abort_flag, p.dev_error, p.wait_cycles, 0x311);
+            // Issue order per tile e: Q_0 K^T (e), P_1 V (e-1), Q_1 K^T (e), P_0 V (e).
+            // S_h(e) overwrites P_h(e-1) in TMEM; the P.V reading it was issued
+            // earlier by this warp and the tensor pipe runs one issuer's MMAs in
+            // issue order, so no wait separates them.
+            bool ok = warp_wait(&bars[B_QREADY0], 0, abort_flag, p.dev_error, p.wait_cycles, 0x311);
             tc_fence_after();
             for (int e = 0; e < NE && ok; ++e) {
                 const int sk = e % NSK, uk = e / NSK, sv = e % NSV, uv = e / NSV;
                 if (e == nR && nR > 0) {
                     // Q of phase R is no longer read once every MMA so far completed
-                    umma_commit(&bars[B_QFREE]);
-                    if (!wait_or_abort(&bars[B_QREADY1], 0, abort_flag, p.dev_error, p.wait_cycles, 0x312)) { ok = false; break; }
+                    umma_commit_elect(&bars[B_QFREE]);
+                    if (!warp_wait(&bars[B_QREADY1], 0, abort_flag, p.dev_error, p.wait_cycles, 0x312)) { ok = false; break; }
                 }
-                if (!wait_or_abort(&bars[B_KREADY + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x313)) { ok = false; break; }
-                if (e > 0 && !wait_or_abort(&bars[B_PVDONE + 0], (e - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x314)) { ok = false; break; }
+                if (!warp_wait(&bars[B_KREADY + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x313)) { ok = false; break; }
                 tc_fence_after();
                 qk(0, sk);
                 if (NH == 2) {
                     if (e > 0) {
                         // head 1's P.V of the previous tile runs while head 0's softmax works
                         const int pe = e - 1, psv = pe % NSV, puv = pe / NSV;
-                        if (!wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x315)) { ok = false; break; }
-                        if (!wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x316)) { ok = false; break; }
+                        if (!warp_wait(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x315)) { ok = false; break; }
+                        if (!warp_wait(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x316)) { ok = false; break; }
                         tc_fence_after();
                         pv(1, psv, pe == 0);
-                        umma_commit(&bars[B_VEMPTY + psv]);
-                        if (!wait_or_abort(&bars[B_PVDONE + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x317)) { ok = false; break; }
-                        tc_fence_after();
+                        umma_commit_elect(&bars[B_VEMPTY + psv]);
                     }
                     qk(1, sk);
                 }
-                umma_commit(&bars[B_KEMPTY + sk]);
-                if (!wait_or_abort(&bars[B_PFULL + 0], e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x318)) { ok = false; break; }
-                if (!wait_or_abort(&bars[B_VFULL + sv], uv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x319)) { ok = false; break; }
+                umma_commit_elect(&bars[B_KEMPTY + sk]);
+                if (!warp_wait(&bars[B_PFULL + 0], e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x318)) { ok = false; break; }
+                if (!warp_wait(&bars[B_VFULL + sv], uv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x319)) { ok = false; break; }
                 tc_fence_after();
                 pv(0, sv, e == 0);
-                if (NH == 1) umma_commit(&bars[B_VEMPTY + sv]);
+                if (NH == 1) umma_commit_elect(&bars[B_VEMPTY + sv]);
             }
             if (ok && NH == 2 && NE > 0) {
                 const int pe = NE - 1, psv = pe % NSV, puv = pe / NSV;
-                if (wait_or_abort(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31a) &&
-                    wait_or_abort(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31b)) {
+                if (warp_wait(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31a) &&
+                    warp_wait(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31b)) {
                     tc_fence_after();
                     pv(1, psv, pe == 0);
-                    umma_commit(&bars[B_VEMPTY + psv]);
+                    umma_commit_elect(&bars[B_VEMPTY + psv]);
                 }
             }
-            // drain: every MMA issued by this thread completed before TMEM is released
-            umma_commit(&bars[B_DRAIN]);
+            // drain: every MMA issued by this warp completed before TMEM is released
+            umma_commit_elect(&bars[B_DRAIN]);
             mbar_wait(&bars[B_DRAIN], 0);
         }
     } else if (warp < 8) {

@@ -83,32 +83,6 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- MMA
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// A from tensor memory: D[tmem] (+)= A[tmem] * B[smem]^T (kind::f16).  The A
-// tile (M = 128 rows = lanes, K = 16) occupies 8 consecutive 32-bit columns,
-// two 16-bit elements per column (even k in the low half).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Warpgroup register reallocation (all four warps of a warpgroup execute it).
 template <int N> __device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 template <int N> __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
@@ -152,14 +126,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b)
     return d;
 }
 
-// Arrive on `bar` once every tcgen05 operation issued so far by this thread completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-
 // ---------------------------------------------------------------- CTA pairs
 // The cta_group::2 forms: one MMA spans the two CTAs of a cluster pair.  Rows
 // [0, 128) of A and of D live in CTA 0 (its shared memory / TMEM), rows
@@ -180,70 +146,12 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Arrive on the mbarrier at `bar`'s offset in both CTAs of the pair once every
-// pair MMA issued so far by this thread completed.
-__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"((unsigned short)0x3)
-        : "memory");
-}
-// Arrive on this CTA's `bar` only.
-__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar)
-{
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// Warp-collective forms of the pair MMA and commits: the whole (converged)
-// warp executes them with warp-uniform operands and one lane, chosen by
-// elect.sync, issues the instruction.  Keeping the issuing loop on a full warp
-// lets the descriptors live in uniform registers; a single divergent thread
-// pays a per-instruction detour to make its operands uniform.
-__device__ __forceinline__ void umma_pair_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                   uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_pair_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                   uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
+// Warp-collective MMA issue and commits: the whole (converged) warp executes
+// them with warp-uniform operands and one lane, chosen by elect.sync, issues
+// the instructions.  Keeping the issuing loop on a full warp lets the
+// descriptors live in uniform registers; a single divergent thread pays a
+// per-instruction detour to make its operands uniform.  Commits of the pair
+// kernel:
 __device__ __forceinline__ void umma_commit_pair_both_elect(uint64_t* bar)
 {
     asm volatile(
@@ -260,6 +168,131 @@ __device__ __forceinline__ void umma_commit_pair_local_elect(uint64_t* bar)
         "{\n\t.reg .pred e;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+// A whole K = 128 reduction as eight pair MMAs from one elected lane, with
+// the descriptors of steps 1..7 made by adding immediates to the start-address
+// field of step 0's (descriptor units of 16 bytes; every address stays below
+// 2^18 bytes, so the 14-bit field never carries).  Q K^T: A = a 128-row
+// K-major tile of two 64-column atoms (step k at (k / 4) * 1024 + (k % 4) * 2
+// units), B = a 64-row K-major tile of two atoms (step k at (k / 4) * 512 +
+// (k % 4) * 2); the first step overwrites D unless `acc0`.
+__device__ __forceinline__ void umma_pair_qk_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t acc0)
+{
+    const uint32_t alo = (uint32_t)a_desc, ahi = (uint32_t)(a_desc >> 32);
+    const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);
+#define JL_QK_STEP(AO, BO)                                                                     \
+    "add.u32 al, %1, " #AO ";\n\tadd.u32 bl, %3, " #BO ";\n\t"                              \
+    "mov.b64 da, {al, %2};\n\tmov.b64 db, {bl, %4};\n\t"                                    \
+    "@e tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, t;\n\t"
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "setp.eq.b32 t, %6, %6;\n\t"
+        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, p;\n\t"
+        JL_QK_STEP(2, 2) JL_QK_STEP(4, 4) JL_QK_STEP(6, 6)
+        JL_QK_STEP(1024, 512) JL_QK_STEP(1026, 514) JL_QK_STEP(1028, 516) JL_QK_STEP(1030, 518)
+        "}" ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
+#undef JL_QK_STEP
+}
+
+// P V over a 128-key tile as eight pair MMAs from one elected lane: A = P in
+// tensor memory (step k at column a_tmem + 8 k), B = an MN-major V tile whose
+// K = 16 slices lie 2048 bytes apart (128 descriptor units); the first step
+// overwrites D unless `acc0`.
+__device__ __forceinline__ void umma_pair_pv_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t acc0)
+{
+    const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);
+#define JL_PV_STEP(AO, BO)                                                                     \
+    "add.u32 ta, %1, " #AO ";\n\tadd.u32 bl, %2, " #BO ";\n\t"                              \
+    "mov.b64 db, {bl, %3};\n\t"                                                              \
+    "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ta], db, %4, t;\n\t"
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 ta, bl;\n\t.reg .b64 db;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 t, %5, %5;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], db, %4, p;\n\t"
+        JL_PV_STEP(8, 128) JL_PV_STEP(16, 256) JL_PV_STEP(24, 384) JL_PV_STEP(32, 512)
+        JL_PV_STEP(40, 640) JL_PV_STEP(48, 768) JL_PV_STEP(56, 896)
+        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
+#undef JL_PV_STEP
+}
+
+// The one-CTA forms (cta_group::1): Q K^T with A and B both 128-row K-major
+// tiles (atoms 1024 units apart; D = 64 has one atom, four steps) and P V as
+// in umma_pair_pv_k128.
+#define JL_MMA1 "@e tcgen05.mma.cta_group::1.kind::f16 "
+__device__ __forceinline__ void umma_qk_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc)
+{
+    const uint32_t alo = (uint32_t)a_desc, ahi = (uint32_t)(a_desc >> 32);
+    const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);
+#define JL_QK1_STEP(O)                                                                          \
+    "add.u32 al, %1, " #O ";\n\tadd.u32 bl, %3, " #O ";\n\t"                                 \
+    "mov.b64 da, {al, %2};\n\tmov.b64 db, {bl, %4};\n\t" JL_MMA1 "[%0], da, db, %5, t;\n\t"
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %5, %5;\n\t"
+        "setp.eq.b32 t, %5, %5;\n\t"
+        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t" JL_MMA1 "[%0], da, db, %5, p;\n\t"
+        JL_QK1_STEP(2) JL_QK1_STEP(4) JL_QK1_STEP(6)
+        JL_QK1_STEP(1024) JL_QK1_STEP(1026) JL_QK1_STEP(1028) JL_QK1_STEP(1030)
+        "}" ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_qk_k64(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc)
+{
+    const uint32_t alo = (uint32_t)a_desc, ahi = (uint32_t)(a_desc >> 32);
+    const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %5, %5;\n\t"
+        "setp.eq.b32 t, %5, %5;\n\t"
+        "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t" JL_MMA1 "[%0], da, db, %5, p;\n\t"
+        JL_QK1_STEP(2) JL_QK1_STEP(4) JL_QK1_STEP(6)
+        "}" ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc)
+        : "memory");
+#undef JL_QK1_STEP
+}
+__device__ __forceinline__ void umma_pv_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t acc0)
+{
+    const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);
+#define JL_PV1_STEP(AO, BO)                                                                     \
+    "add.u32 ta, %1, " #AO ";\n\tadd.u32 bl, %2, " #BO ";\n\t"                               \
+    "mov.b64 db, {bl, %3};\n\t" JL_MMA1 "[%0], [ta], db, %4, t;\n\t"
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 ta, bl;\n\t.reg .b64 db;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "setp.eq.b32 t, %5, %5;\n\t"
+        "mov.b64 db, {%2, %3};\n\t" JL_MMA1 "[%0], [%1], db, %4, p;\n\t"
+        JL_PV1_STEP(8, 128) JL_PV1_STEP(16, 256) JL_PV1_STEP(24, 384) JL_PV1_STEP(32, 512)
+        JL_PV1_STEP(40, 640) JL_PV1_STEP(48, 768) JL_PV1_STEP(56, 896)
+        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)
+        : "memory");
+#undef JL_PV1_STEP
+}
+#undef JL_MMA1
+
+// Arrive on `bar` once every tcgen05 operation this warp's elected lanes
+// issued so far completed (one-CTA kernels, warp-collective).
+__device__ __forceinline__ void umma_commit_elect(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
         : "memory");
 }
 
