@@ -48,7 +48,7 @@ enum {
     P_QFULL = 0, P_QREADY0, P_QREADY1, P_QFREE,
     P_KFULL, P_KREADY = P_KFULL + NS, P_KEMPTY = P_KREADY + NS,
     P_VFULL = P_KEMPTY + NS, P_VPEER = P_VFULL + NS, P_VEMPTY = P_VPEER + NS,
-    P_SFULL = P_VEMPTY + NS, P_PFULL = P_SFULL + 2, P_PVDONE = P_PFULL + 2,
+    P_SFULL = P_VEMPTY + NS, P_PFULL = P_SFULL + 2, P_PVDONE = P_PFULL + 4,
     P_DRAIN = P_PVDONE + 2, P_NBARS
 };
 
@@ -105,7 +105,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&bars[P_SFULL + h], 1);
-            mbar_init(&bars[P_PFULL + h], 8);
+            mbar_init(&bars[P_PFULL + 2 * h], 8);      // first half of P_h
+            mbar_init(&bars[P_PFULL + 2 * h + 1], 8);  // second half
             mbar_init(&bars[P_PVDONE + h], 1);
         }
         mbar_init(&bars[P_DRAIN], 1);
@@ -185,18 +186,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 umma_pair_qk_k128(tm + h * 128, sdesc_sw128(qaddr, 16, 1024), sdesc_sw128(kaddr, 16, 1024), IDESC_QK, 0u);
                 umma_commit_pair_both_elect(&bars[P_SFULL + h]);
             };
-            auto pv = [&](int h, int s, bool first) {
-                const uint32_t vaddr = sbase + S::V0 + s * S::VTILE;
-                umma_pair_pv_k128(tm + 256 + h * 128, tm + h * 128, sdesc_sw128(vaddr, S::VTILE, 1024), IDESC_PV,
-                                  first ? 0u : 1u);
-                umma_commit_pair_both_elect(&bars[P_PVDONE + h]);
-            };
-            // V half of tile pe landed in both CTAs and P_h of tile pe is in both TMEMs
-            auto pv_ready = [&](int h, int pe) {
+            // P_h V of tile pe, issued half by half as the softmax publishes the
+            // halves of P_h (V's halves landed in both CTAs: checked for head 0)
+            auto pv = [&](int h, int pe) {
                 const int s = pe % NS, u = pe / NS;
-                return warp_wait<true>(&bars[P_PFULL + h], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x411 + h) &&
-                       (h == 1 || (warp_wait(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x413) &&
-                                   warp_wait<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x414)));
+                if (h == 0 && !(warp_wait(&bars[P_VFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x413) &&
+                                warp_wait<true>(&bars[P_VPEER + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x414)))
+                    return false;
+                const uint64_t vdesc = sdesc_sw128(sbase + S::V0 + s * S::VTILE, S::VTILE, 1024);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (!warp_wait<true>(&bars[P_PFULL + 2 * h + half], pe & 1, abort_flag, p.dev_error, p.wait_cycles,
+                                         0x411 + h))
+                        return false;
+                    tc_fence_after();
+                    umma_pair_pv_k64(tm + 256 + h * 128, tm + h * 128 + 32 * half, vdesc + 512 * half, IDESC_PV,
+                                     (pe == 0 && half == 0) ? 0u : 1u);
+                }
+                umma_commit_pair_both_elect(&bars[P_PVDONE + h]);
+                return true;
             };
             // Issue order per tile e: P_0 V (tile e-1), Q_0 K^T (tile e), P_1 V
             // (tile e-1), Q_1 K^T (tile e).  S_h(e) overwrites P_h(e-1) in TMEM;
@@ -206,11 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             tc_fence_after();
             for (int e = 0; e < NE && ok; ++e) {
                 const int s = e % NS, u = e / NS, pe = e - 1, ps = (e + NS - 1) % NS;
-                if (e > 0) {
-                    if (!pv_ready(0, pe)) { ok = false; break; }
-                    tc_fence_after();
-                    pv(0, ps, pe == 0);
-                }
+                if (e > 0 && !pv(0, pe)) { ok = false; break; }
                 if (e == nR && nR > 0) {
                     // Q of phase R is no longer read once every MMA so far completed
                     umma_commit_pair_both_elect(&bars[P_QFREE]);
@@ -220,9 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 qk(0, s);
                 if (e > 0) {
-                    if (!pv_ready(1, pe)) { ok = false; break; }
-                    tc_fence_after();
-                    pv(1, ps, pe == 0);
+                    if (!pv(1, pe)) { ok = false; break; }
                     umma_commit_pair_both_elect(&bars[P_VEMPTY + ps]);
                 }
                 qk(1, s);
@@ -230,15 +232,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
             if (ok && NE > 0) {
                 const int pe = NE - 1, ps = pe % NS;
-                if (pv_ready(0, pe)) {
-                    tc_fence_after();
-                    pv(0, ps, pe == 0);
-                    if (pv_ready(1, pe)) {
-                        tc_fence_after();
-                        pv(1, ps, pe == 0);
-                        umma_commit_pair_both_elect(&bars[P_VEMPTY + ps]);
-                    }
-                }
+                if (pv(0, pe) && pv(1, pe)) umma_commit_pair_both_elect(&bars[P_VEMPTY + ps]);
             }
             // drain: every MMA issued by this warp completed before the pair
             // meets at the closing cluster barrier
@@ -305,10 +299,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // -------------------------------------------------------------- softmax (head hh)
         const int hh = (warp - 8) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        const uint32_t pfull = lead(P_PFULL + hh);
+        const uint32_t pfull = lead(P_PFULL + 2 * hh);
         softmax_role<D, true>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128, lane_base + 256 + hh * 128,
-                              &bars[P_SFULL + hh], &bars[P_PVDONE + hh], [pfull] { mbar_arrive_cluster(pfull); },
-                              abort_flag);
+                              &bars[P_SFULL + hh], &bars[P_PVDONE + hh],
+                              [pfull](int half) { mbar_arrive_cluster(pfull + 8u * (uint32_t)half); }, abort_flag);
     }
     tc_fence_before();
     __syncthreads();

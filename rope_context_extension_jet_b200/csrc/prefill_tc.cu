@@ -52,7 +52,7 @@ enum {
     B_QFULL = 0, B_QREADY0, B_QREADY1, B_QFREE,
     B_KFULL, B_KREADY = B_KFULL + NSK, B_KEMPTY = B_KREADY + NSK,
     B_VFULL = B_KEMPTY + NSK, B_VEMPTY = B_VFULL + NSV,
-    B_SFULL = B_VEMPTY + NSV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
+    B_SFULL = B_VEMPTY + NSV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 4,
     B_DRAIN = B_PVDONE + 2, NBARS
 };
 
@@ -106,7 +106,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&bars[B_SFULL + h], 1);
-            mbar_init(&bars[B_PFULL + h], 4);
+            mbar_init(&bars[B_PFULL + 2 * h], 4);      // first half of P_h
+            mbar_init(&bars[B_PFULL + 2 * h + 1], 4);  // second half
             mbar_init(&bars[B_PVDONE + h], 1);
         }
         mbar_init(&bars[B_DRAIN], 1);
@@ -181,10 +182,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     umma_qk_k64(tm + h * 128, a, bk, IDESC_QK);
                 umma_commit_elect(&bars[B_SFULL + h]);
             };
-            auto pv = [&](int h, int sv, bool first) {
-                umma_pv_k128(tm + 256 + h * 128, tm + h * 128, sdesc_sw128(sbase + S::V0 + sv * S::TILE, ATOM, 1024),
-                             IDESC_PV, first ? 0u : 1u);
+            // P_h V of tile pe (V in stage sv), issued half by half as the
+            // softmax publishes the halves of P_h
+            auto pv = [&](int h, int pe, int sv, int code) {
+                const uint64_t vdesc = sdesc_sw128(sbase + S::V0 + sv * S::TILE, ATOM, 1024);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (!warp_wait(&bars[B_PFULL + 2 * h + half], pe & 1, abort_flag, p.dev_error, p.wait_cycles, code))
+                        return false;
+                    tc_fence_after();
+                    umma_pv_k64(tm + 256 + h * 128, tm + h * 128 + 32 * half, vdesc + 512 * half, IDESC_PV,
+                                (pe == 0 && half == 0) ? 0u : 1u);
+                }
                 umma_commit_elect(&bars[B_PVDONE + h]);
+                return true;
             };
             // Issue order per tile e: Q_0 K^T (e), P_1 V (e-1), Q_1 K^T (e), P_0 V (e).
             // S_h(e) overwrites P_h(e-1) in TMEM; the P.V reading it was issued
@@ -206,29 +217,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (e > 0) {
                         // head 1's P.V of the previous tile runs while head 0's softmax works
                         const int pe = e - 1, psv = pe % NSV, puv = pe / NSV;
-                        if (!warp_wait(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x315)) { ok = false; break; }
                         if (!warp_wait(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x316)) { ok = false; break; }
-                        tc_fence_after();
-                        pv(1, psv, pe == 0);
+                        if (!pv(1, pe, psv, 0x315)) { ok = false; break; }
                         umma_commit_elect(&bars[B_VEMPTY + psv]);
                     }
                     qk(1, sk);
                 }
                 umma_commit_elect(&bars[B_KEMPTY + sk]);
-                if (!warp_wait(&bars[B_PFULL + 0], e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x318)) { ok = false; break; }
                 if (!warp_wait(&bars[B_VFULL + sv], uv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x319)) { ok = false; break; }
-                tc_fence_after();
-                pv(0, sv, e == 0);
+                if (!pv(0, e, sv, 0x318)) { ok = false; break; }
                 if (NH == 1) umma_commit_elect(&bars[B_VEMPTY + sv]);
             }
             if (ok && NH == 2 && NE > 0) {
                 const int pe = NE - 1, psv = pe % NSV, puv = pe / NSV;
-                if (warp_wait(&bars[B_PFULL + 1], pe & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31a) &&
-                    warp_wait(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31b)) {
-                    tc_fence_after();
-                    pv(1, psv, pe == 0);
+                if (warp_wait(&bars[B_VFULL + psv], puv & 1, abort_flag, p.dev_error, p.wait_cycles, 0x31b) &&
+                    pv(1, pe, psv, 0x31a))
                     umma_commit_elect(&bars[B_VEMPTY + psv]);
-                }
             }
             // drain: every MMA issued by this warp completed before TMEM is released
             umma_commit_elect(&bars[B_DRAIN]);
@@ -288,10 +292,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int hh = (warp - 8) >> 2;
         if (hh < NH) {
             const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-            uint64_t* pfull = &bars[B_PFULL + hh];
+            uint64_t* pfull = &bars[B_PFULL + 2 * hh];
             softmax_role<D, false>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128,
                                    lane_base + 256 + hh * 128, &bars[B_SFULL + hh], &bars[B_PVDONE + hh],
-                                   [pfull] { mbar_arrive(pfull); }, abort_flag);
+                                   [pfull](int half) { mbar_arrive(pfull + half); }, abort_flag);
         }
     }
     tc_fence_before();

@@ -249,7 +249,8 @@ __device__ __forceinline__ void rope_steps(int t, const TcParams& p, float (&stc
 // warps.  For each key tile e: wait for S = Q K^T in TMEM (`sfull`), apply the
 // causal / length / band masks, online softmax in base 2 with lazy O rescaling
 // (after the previous P.V finished, `pvdone`), write P (bf16) over the first 64
-// columns of S and signal the MMA issuer (`arrive_p`); finally O / l -> out.
+// columns of S in two halves of 64 keys, signalling the MMA issuer after each
+// (`arrive_p(half)`); finally O / l -> out.
 // s_col / o_col are this warp's TMEM addresses of S and O.
 template <int D, bool CLUSTER, class ArriveP>
 __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& tp, int qb, int head, int b,
@@ -321,29 +322,37 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
         }
         const float ms = m_used == -INFINITY ? 0.f : m_used;
         // p = 2^(x * scale * log2(e) - m), two columns per packed instruction
+        // P in two halves of BN / 2 keys, each published (arrive_p(half)) as soon
+        // as it is in TMEM, so P.V of the first half overlaps the exponentials of
+        // the second
         const float2 sl = make_float2(sl2, sl2), nm = make_float2(-ms, -ms);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint32_t pk[BN / 2];
 #pragma unroll
-        for (int u = 0; u < BN; u += 4) {
-            const float2 y0 = fma2(make_float2(x[u], x[u + 1]), sl, nm);
-            const float2 y1 = fma2(make_float2(x[u + 2], x[u + 3]), sl, nm);
-            const float2 p0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-            const float2 p1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-            acc0 = add2(acc0, p0);
-            acc1 = add2(acc1, p1);
-            pk[u >> 1] = pack_bf16x2(p0.x, p0.y);
-            pk[(u >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
-        }
-        l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        // The previous P.V of this head has finished: the MMA issuer issues it
-        // before Q K^T of this tile, whose commit (sfull) tracks every earlier
-        // MMA of that thread.  So P may overwrite its columns now; the rare O
-        // rescale still checks pvdone explicitly.
-        if (e > 0 && __any_sync(0xffffffffu, resc)) {
-            if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x332)) { ok = false; break; }
-            tc_fence_after();
-            {
+        for (int half = 0; half < 2; ++half) {
+            uint32_t pk[BN / 4];
+#pragma unroll
+            for (int v = 0; v < BN / 2; v += 4) {
+                const int u = half * (BN / 2) + v;
+                const float2 y0 = fma2(make_float2(x[u], x[u + 1]), sl, nm);
+                const float2 y1 = fma2(make_float2(x[u + 2], x[u + 3]), sl, nm);
+                const float2 p0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+                const float2 p1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+                acc0 = add2(acc0, p0);
+                acc1 = add2(acc1, p1);
+                pk[v >> 1] = pack_bf16x2(p0.x, p0.y);
+                pk[(v >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+            }
+            // The previous P.V of this head has finished: the MMA issuer issues
+            // it before Q K^T of this tile, whose commit (sfull) tracks every
+            // earlier MMA of that thread.  So P may overwrite its columns now;
+            // the rare O rescale (before any of this tile's P is published, so
+            // before this tile's P.V) still checks pvdone explicitly.
+            if (half == 0 && e > 0 && __any_sync(0xffffffffu, resc)) {
+                if (!warp_wait<CLUSTER>(pvdone, (e - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x332)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t tt[32];
@@ -354,18 +363,15 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
                     tmem_st32(o_col + cc * 32, tt);
                 }
             }
+            static_assert(BN / 4 == 32, "one 32-column TMEM store per half");
+            tmem_st32(s_col + half * 32, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_p(half);
         }
-#pragma unroll
-        for (int cc = 0; cc < BN / 64; ++cc) {
-            uint32_t tt[32];
-#pragma unroll
-            for (int u = 0; u < 32; ++u) tt[u] = pk[cc * 32 + u];
-            tmem_st32(s_col + cc * 32, tt);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_p();
+        if (!ok) break;
+        l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
     }
     // epilogue: O / l -> bf16 -> out
     if (ok && NE > 0 && warp_wait<CLUSTER>(pvdone, (NE - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x333)) {

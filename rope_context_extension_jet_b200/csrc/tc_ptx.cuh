@@ -296,6 +296,37 @@ __device__ __forceinline__ void umma_commit_elect(uint64_t* bar)
         : "memory");
 }
 
+// Half of a P V: the four pair (cta_group::2) or one-CTA MMAs over 64 keys,
+// A = P in tensor memory (step k at a_tmem + 8 k), B = V slices 128 descriptor
+// units apart; the first step overwrites D unless `acc0`.  The second half of a
+// tile is the same call at a_tmem + 32 and b_desc + 512.
+#define JL_PVH(CG)                                                                                          \
+    {                                                                                                       \
+        const uint32_t blo = (uint32_t)b_desc, bhi = (uint32_t)(b_desc >> 32);                              \
+        asm volatile(                                                                                       \
+            "{\n\t.reg .pred p, t, e;\n\t.reg .b32 ta, bl;\n\t.reg .b64 db;\n\t"                      \
+            "elect.sync _|e, 0xffffffff;\n\t"                                                               \
+            "setp.ne.b32 p, %5, 0;\n\t"                                                                     \
+            "setp.eq.b32 t, %5, %5;\n\t"                                                                    \
+            "mov.b64 db, {%2, %3};\n\t"                                                                     \
+            "@e tcgen05.mma.cta_group::" CG ".kind::f16 [%0], [%1], db, %4, p;\n\t"                       \
+            "add.u32 ta, %1, 8;\n\tadd.u32 bl, %2, 128;\n\tmov.b64 db, {bl, %3};\n\t"                    \
+            "@e tcgen05.mma.cta_group::" CG ".kind::f16 [%0], [ta], db, %4, t;\n\t"                       \
+            "add.u32 ta, %1, 16;\n\tadd.u32 bl, %2, 256;\n\tmov.b64 db, {bl, %3};\n\t"                   \
+            "@e tcgen05.mma.cta_group::" CG ".kind::f16 [%0], [ta], db, %4, t;\n\t"                       \
+            "add.u32 ta, %1, 24;\n\tadd.u32 bl, %2, 384;\n\tmov.b64 db, {bl, %3};\n\t"                   \
+            "@e tcgen05.mma.cta_group::" CG ".kind::f16 [%0], [ta], db, %4, t;\n\t"                       \
+            "}" ::"r"(d_tmem), "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc0)                        \
+            : "memory");                                                                                    \
+    }
+__device__ __forceinline__ void umma_pair_pv_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t acc0)
+JL_PVH("2")
+__device__ __forceinline__ void umma_pv_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t acc0)
+JL_PVH("1")
+#undef JL_PVH
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 //   bits [0,14) start address >> 4; [16,30) leading byte offset >> 4;
 //   [32,46) stride byte offset >> 4; [46,48) version = 1; [49,52) base offset = 0;
