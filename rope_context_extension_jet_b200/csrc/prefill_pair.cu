@@ -250,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         regs_dec<72>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
-        float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
+        float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
         // operand scales of this call (powers of two, see range_exp)
         const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
@@ -259,10 +259,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (ok) {
             for (int h = 0; h < 2; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                    rotate_tile<D, BM, true, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
                                              sts, lq);
                 else
-                    rotate_tile<D, BM, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
+                    rotate_tile<D, BM, true, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -275,7 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
                 if (!warp_wait<true>(&bars[P_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x432)) { ok = false; break; }
                 for (int h = 0; h < 2; ++h)
-                    rotate_tile<D, BM, false>(smem + h * S::QTILE, t, p,
+                    rotate_tile<D, BM, false, true>(smem + h * S::QTILE, t, p,
                                               [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -285,9 +285,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
             unsigned char* kt = smem + S::K0 + s * S::KTILE;
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts, lk);
+                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts, lk);
             else
-                rotate_tile<D, KROWS, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
+                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
             fence_proxy_async_smem();
             __syncwarp();
             // (test hook: the first key tile is never released, so the MMA warp's

@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         regs_dec<88>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
-        float stc[8], sts[8];  // per-frequency one-position step R(theta_m)
+        float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
         // operand scales of this call (powers of two, see range_exp)
         const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
@@ -251,10 +251,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok) {
             for (int h = 0; h < NH; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                    rotate_tile<D, BM, true, false>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
                                              sts, lq);
                 else
-                    rotate_tile<D, BM, true>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
+                    rotate_tile<D, BM, true, false>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
                 if (!warp_wait(&bars[B_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x322)) { ok = false; break; }
                 for (int h = 0; h < NH; ++h)
-                    rotate_tile<D, BM, false>(smem + h * S::TILE, t, p,
+                    rotate_tile<D, BM, false, false>(smem + h * S::TILE, t, p,
                                           [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -276,10 +276,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x323)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN);
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc,
+                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc,
                                          sts, lk);
             else
-                rotate_tile<D, BM, true>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
+                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
             fence_proxy_async_smem();
             __syncwarp();
             // (test hook: the first key tile is never released, so the MMA

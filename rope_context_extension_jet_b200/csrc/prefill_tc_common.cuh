@@ -174,23 +174,35 @@ __device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__usho
 // floor(j/G) and i - floor(i/G)); the angles of the first row come from the
 // exact fixed-point phase, later rows advance by the per-frequency step
 // rotation R(theta_m) (any other step is recomputed exactly).
-template <int D, int ROWS, bool IN_BF16, class PosFn>
+//
+// PACKED: the arithmetic runs on frequency pairs with packed f32x2 FMAs (fewer
+// issue slots: the CTA-pair kernel, whose rotation warps compete with the
+// softmax warps for issue); otherwise on scalar FMAs (the one-CTA kernel, which
+// measured faster that way).  Both compute in fp32, each value as one product
+// and one fused multiply-add.
+template <int D, int ROWS, bool IN_BF16, bool PACKED, class PosFn>
 __device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const TcParams& p, PosFn pos,
-                                            const float (&stc)[8], const float (&sts)[8], float lam)
+                                            const float2 (&stc)[4], const float2 (&sts)[4], float lam)
 {
     constexpr int H = D / 2, CH = H / 8, RPT = ROWS * CH / 128;  // 128 threads = CH chunks x (ROWS / RPT) row groups
     static_assert(RPT >= 1 && ROWS * CH == 128 * RPT, "rotation thread mapping");
     const int c = t % CH, row0 = (t / CH) * RPT;
-    // (cs, sn) carry the operand scale lam: the step rotation is linear, so
-    // every row it produces keeps it
-    float cs[8], sn[8];
-    uint32_t prev = pos(row0);
+    // cos / sin of the thread's 8 frequencies as 4 pairs (2w, 2w + 1).  (cs, sn)
+    // carry the operand scale lam: the step rotation is linear, so every row it
+    // produces keeps it.
+    float2 cs[4], sn[4];
+    auto exact = [&](uint32_t q) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        rope_cs_fast(prev, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
-        cs[u] *= lam;
-        sn[u] *= lam;
-    }
+        for (int w = 0; w < 4; ++w) {
+            float c0, s0, c1, s1;
+            rope_cs_fast(q, p.turns.hi[c * 8 + 2 * w], p.turns.lo[c * 8 + 2 * w], c0, s0);
+            rope_cs_fast(q, p.turns.hi[c * 8 + 2 * w + 1], p.turns.lo[c * 8 + 2 * w + 1], c1, s1);
+            cs[w] = make_float2(c0 * lam, c1 * lam);
+            sn[w] = make_float2(s0 * lam, s1 * lam);
+        }
+    };
+    uint32_t prev = pos(row0);
+    exact(prev);
 #pragma unroll 2
     for (int s = 0; s < RPT; ++s) {
         const int r = row0 + s;
@@ -198,18 +210,22 @@ __device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const Tc
             const uint32_t cur = pos(r);
             if (cur == prev + 1) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float c2 = cs[u] * stc[u] - sn[u] * sts[u];
-                    sn[u] = sn[u] * stc[u] + cs[u] * sts[u];
-                    cs[u] = c2;
+                for (int w = 0; w < 4; ++w) {
+                    // (c, s) <- (c cos t - s sin t, s cos t + c sin t)
+                    if (PACKED) {
+                        const float2 c2 = __ffma2_rn(make_float2(-sn[w].x, -sn[w].y), sts[w], __fmul2_rn(cs[w], stc[w]));
+                        sn[w] = __ffma2_rn(cs[w], sts[w], __fmul2_rn(sn[w], stc[w]));
+                        cs[w] = c2;
+                    } else {
+                        const float2 c2 = make_float2(cs[w].x * stc[w].x - sn[w].x * sts[w].x,
+                                                      cs[w].y * stc[w].y - sn[w].y * sts[w].y);
+                        sn[w] = make_float2(sn[w].x * stc[w].x + cs[w].x * sts[w].x,
+                                            sn[w].y * stc[w].y + cs[w].y * sts[w].y);
+                        cs[w] = c2;
+                    }
                 }
             } else if (cur != prev) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    rope_cs_fast(cur, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], cs[u], sn[u]);
-                    cs[u] *= lam;
-                    sn[u] *= lam;
-                }
+                exact(cur);
             }
             prev = cur;
         }
@@ -221,28 +237,38 @@ __device__ __forceinline__ void rotate_tile(unsigned char* tile, int t, const Tc
         uint32_t oa[4], ob[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            float x0, x1, y0, y1;
-            if (IN_BF16) {
-                x0 = bf16_lo(la[w]); x1 = bf16_hi(la[w]); y0 = bf16_lo(lb[w]); y1 = bf16_hi(lb[w]);
+            // x = the pair's first members (dims m, m + 1), y = their partners (m + d/2, ...)
+            const float2 x = IN_BF16 ? make_float2(bf16_lo(la[w]), bf16_hi(la[w])) : make_float2(f16_lo(la[w]), f16_hi(la[w]));
+            const float2 y = IN_BF16 ? make_float2(bf16_lo(lb[w]), bf16_hi(lb[w])) : make_float2(f16_lo(lb[w]), f16_hi(lb[w]));
+            if (PACKED) {
+                const float2 lo = __ffma2_rn(make_float2(-y.x, -y.y), sn[w], __fmul2_rn(x, cs[w]));  // x c - y s
+                const float2 hi = __ffma2_rn(y, cs[w], __fmul2_rn(x, sn[w]));                       // x s + y c
+                oa[w] = pack_f16x2(lo.x, lo.y);
+                ob[w] = pack_f16x2(hi.x, hi.y);
             } else {
-                x0 = f16_lo(la[w]); x1 = f16_hi(la[w]); y0 = f16_lo(lb[w]); y1 = f16_hi(lb[w]);
+                oa[w] = pack_f16x2(x.x * cs[w].x - y.x * sn[w].x, x.y * cs[w].y - y.y * sn[w].y);
+                ob[w] = pack_f16x2(x.x * sn[w].x + y.x * cs[w].x, x.y * sn[w].y + y.y * cs[w].y);
             }
-            const int u0 = 2 * w, u1 = 2 * w + 1;
-            oa[w] = pack_f16x2(x0 * cs[u0] - y0 * sn[u0], x1 * cs[u1] - y1 * sn[u1]);
-            ob[w] = pack_f16x2(x0 * sn[u0] + y0 * cs[u0], x1 * sn[u1] + y1 * cs[u1]);
         }
         *plo = make_uint4(oa[0], oa[1], oa[2], oa[3]);
         *phi = make_uint4(ob[0], ob[1], ob[2], ob[3]);
     }
 }
 
-// Per-frequency one-position step rotation R(theta_m) of rotation thread t.
+// Per-frequency one-position step rotation R(theta_m) of rotation thread t, as
+// the 4 frequency pairs rotate_tile works on.
 template <int D>
-__device__ __forceinline__ void rope_steps(int t, const TcParams& p, float (&stc)[8], float (&sts)[8])
+__device__ __forceinline__ void rope_steps(int t, const TcParams& p, float2 (&stc)[4], float2 (&sts)[4])
 {
     const int c = t % (D / 16);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) rope_cs_fast(1u, p.turns.hi[c * 8 + u], p.turns.lo[c * 8 + u], stc[u], sts[u]);
+    for (int w = 0; w < 4; ++w) {
+        float c0, s0, c1, s1;
+        rope_cs_fast(1u, p.turns.hi[c * 8 + 2 * w], p.turns.lo[c * 8 + 2 * w], c0, s0);
+        rope_cs_fast(1u, p.turns.hi[c * 8 + 2 * w + 1], p.turns.lo[c * 8 + 2 * w + 1], c1, s1);
+        stc[w] = make_float2(c0, c1);
+        sts[w] = make_float2(s0, s1);
+    }
 }
 
 // Softmax role of one query head: one thread per query row (= TMEM lane), 4
