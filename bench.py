@@ -78,10 +78,13 @@ PREFILL_KERNEL = "prefill_pair_kernel"
 PREFILL_SOURCES = ("prefill_pair.cu", "prefill_tc_common.cuh", "tc_ptx.cuh", "jl_ptx.cuh", "jl_common.cuh")
 
 
-def prefill_source_hash():
+DECODE_SOURCES = ("decode.cu", "jl_ptx.cuh", "jl_common.cuh")
+
+
+def prefill_source_hash(names=PREFILL_SOURCES):
     import hashlib
     h = hashlib.sha256()
-    for name in PREFILL_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "rope_context_extension_jet_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -365,6 +368,54 @@ def parse_ncu_csv(text):
     return rows
 
 
+# Counters kept from a --set full capture (the rest of its ~1000 stay in the
+# .csv under gpurun_out/)
+NCU_FULL_SHOWN = (
+    "gpu__time_duration.sum", "sm__cycles_elapsed.avg.per_second", "dram__bytes_read.sum",
+    "dram__bytes_write.sum", "dram__cycles_active.avg.pct_of_peak_sustained_elapsed",
+    "gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed",
+    "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active",
+    "sm__inst_executed_pipe_xu.avg.pct_of_peak_sustained_active",
+    "sm__inst_executed_pipe_fma.avg.pct_of_peak_sustained_active",
+    "sm__inst_executed_pipe_alu.avg.pct_of_peak_sustained_active",
+    "sm__inst_executed_pipe_lsu.avg.pct_of_peak_sustained_active",
+    "smsp__issue_active.avg.pct_of_peak_sustained_active", "sm__warps_active.avg.pct_of_peak_sustained_active",
+    "smsp__inst_executed.sum", "launch__registers_per_thread", "launch__grid_size", "launch__cluster_dim_x",
+    "smsp__average_warps_issue_stalled_long_scoreboard_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_wait_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_barrier_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_short_scoreboard_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_math_pipe_throttle_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_mio_throttle_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_lg_throttle_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_no_instruction_per_issue_active.ratio",
+    "smsp__average_warps_issue_stalled_branch_resolving_per_issue_active.ratio",
+    "l1tex__data_pipe_lsu_wavefronts_mem_shared.sum",
+)
+
+
+def parse_ncu_raw_csv(text):
+    """ncu --page raw --csv output (one header row of metric names, one row of
+    units, one row per kernel) as the same dicts as parse_ncu_csv."""
+    import csv
+    import io
+    lines = [ln for ln in text.splitlines() if ln.startswith('"')]
+    recs = list(csv.reader(io.StringIO("\n".join(lines))))
+    if len(recs) < 3:
+        return []
+    head, units = recs[0], recs[1]
+    rows = []
+    for rec in recs[2:]:
+        kname = rec[head.index("Kernel Name")] if "Kernel Name" in head else ""
+        for name, unit, val in zip(head, units, rec):
+            try:
+                v = float(val.replace(",", ""))
+            except ValueError:
+                continue
+            rows.append({"kernel": kname, "id": 0, "metric": name, "unit": unit, "value": v})
+    return rows
+
+
 def launch_summary(rows):
     """Per kernel (name up to its template arguments): launches, total ms, share
     of the summed device time, from gpu__time_duration.sum rows (ns)."""
@@ -393,6 +444,10 @@ def run_ncu(args):
     if args.ncu == "launches":
         bench_args = ["--steps", str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
         extra = ["--metrics", "gpu__time_duration.sum"]
+    elif args.ncu in ("prefill-full", "decode-full"):
+        which = args.ncu.split("-")[0]
+        bench_args = ["--profile", which, "--L", str(args.L), "--steps", "1", "--warmup", "1"]
+        extra = ["--set", "full", "--page", "raw", "-k", "regex:" + NCU_KERNELS[which], "-s", "1", "-c", "1"]
     elif args.ncu == "traffic":
         bench_args = ["--profile", "prefill", "--L", str(args.L), "--steps", "1", "--warmup", "1"]
         extra = ["--metrics", "gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum",
@@ -413,11 +468,10 @@ def run_ncu(args):
     if r.returncode != 0:
         print(r.stdout[-2000:], r.stderr[-2000:])
         raise SystemExit(f"ncu exited {r.returncode}")
-    rows = parse_ncu_csv(open(log).read())
-    shown = " ".join(("'" + c + "'") if ("(" in c or " " in c) else c
-                     for c in ["ncu"] + cmd[1:4] + cmd[6:] if c != sys.executable).replace(
-        os.path.join(ROOT, ""), "")
-    shown = shown.replace(" bench.py", " python bench.py").replace("--log-file", "")
+    text = open(log).read()
+    rows = parse_ncu_raw_csv(text) if args.ncu.endswith("-full") else parse_ncu_csv(text)
+    import shlex
+    shown = shlex.join(["python" if c == sys.executable else c for c in cmd]).replace(os.path.join(ROOT, ""), "")
     lines = []
     if args.ncu == "launches":
         summ = launch_summary(rows)
@@ -432,10 +486,12 @@ def run_ncu(args):
         name = "launches_bench"
     else:
         m = {r["metric"]: r["value"] for r in rows}
+        if args.ncu.endswith("-full"):
+            m = {k: v for k, v in m.items() if any(k.startswith(w) for w in NCU_FULL_SHOWN)}
         dur = m.get("gpu__time_duration.sum", float("nan")) * 1e-9
         dram = m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0)
         rec = {"metrics": m, "seconds": dur, "dram_bytes": dram}
-        if args.ncu in ("prefill", "traffic"):
+        if args.ncu in ("prefill", "traffic", "prefill-full"):
             w = I.C4.with_(L=args.L)
             useful, computed, _, _ = prefill_flops(w)
             rec.update({"workload": f"prefill bf16 B=1 Hq=32 Hkv=8 d=128 L={args.L} G={max(1, -(-args.L // w.w_pretrained))} "
@@ -453,6 +509,8 @@ def run_ncu(args):
         rec["peaks"] = {k: v for k, v in peaks.items()}
         if args.ncu == "traffic":
             name = f"{kname}_L{args.L}_dram"
+        elif args.ncu.endswith("-full"):
+            name = f"{kname}_L{args.L}_full"
         else:
             name = f"{kname}_L{args.L}_counters"
         lines += [f"# `{kname}`: {rec['workload']}", "", "One launch after one warm-up launch (ncu, clock control none),",
@@ -468,7 +526,10 @@ def run_ncu(args):
             lines += ["", f"K/V bytes {rec['kv_bytes']:.4e} over {dur * 1e3:.3f} ms = {rec['gbs_kv']:.0f} GB/s, "
                           f"{rec['frac_of_hbm']:.3f} of the {peaks['source']} HBM copy bandwidth "
                           f"({peaks['hbm_gbs']} GB/s); DRAM counted {dram / 1e9:.3f} GB."]
-    lines += ["", f"Sources: sha256 of the prefill kernel files {prefill_source_hash()[:16]}; "
+    srcs = DECODE_SOURCES if args.ncu.startswith("decode") else PREFILL_SOURCES
+    if args.ncu == "launches":
+        srcs = PREFILL_SOURCES + ("decode.cu", "range_scan.cu")
+    lines += ["", f"Sources: sha256 of {', '.join(srcs)}: {prefill_source_hash(srcs)[:16]}; "
                   f"capture took {secs:.0f} s."]
     prof = os.path.join(ROOT, "profiles")
     with open(os.path.join(prof, name + ".md"), "w") as f:
@@ -498,7 +559,8 @@ def main():
     ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
                     help="run only one kernel on a reduced workload (for ncu captures)")
     ap.add_argument("--L", type=int, default=32768, help="sequence / cache length for --profile")
-    ap.add_argument("--ncu", choices=["launches", "prefill", "decode", "traffic"], default=None,
+    ap.add_argument("--ncu", choices=["launches", "prefill", "decode", "traffic", "prefill-full", "decode-full"],
+                    default=None,
                     help="profiling harness: the bench command (launches), one kernel of the --profile "
                          "workloads (prefill, decode) or one full-size prefill's DRAM bytes (traffic, "
                          "--L 131072), under ncu; writes the summary under profiles/")

@@ -122,3 +122,12 @@ def test_ncu_csv_parsing_and_launch_shares():
     assert (n0, n1) == (1, 2)
     assert t0 == pytest.approx(156.0) and t1 == pytest.approx(2.0)
     assert s0 == pytest.approx(156.0 / 158.0) and s0 + s1 == pytest.approx(1.0)
+
+
+def test_ncu_raw_csv_parsing():
+    text = ('==PROF== noise\n"ID","Kernel Name","gpu__time_duration.sum","dram__bytes_read.sum"\n'
+            '"","","ns","byte"\n"0","prefill_pair_kernel(...)","8,708,000","404,577,000"\n')
+    rows = bench.parse_ncu_raw_csv(text)
+    m = {r["metric"]: r["value"] for r in rows}
+    assert m["gpu__time_duration.sum"] == 8708000.0 and m["dram__bytes_read.sum"] == 404577000.0
+    assert rows[0]["kernel"].startswith("prefill_pair_kernel")
