@@ -768,6 +768,43 @@ def main():
     _, ch_computed, _, _ = prefill_flops(wp, P=P_ch)
     del q_ch, out_ch
 
+    # ---------------- a serving-shaped variable-length batch (jetlong_prefill_varlen):
+    # 64 sequences of seeded lengths in [512, 8192] (Hq=32, Hkv=8, d=128,
+    # w_pretrained=2048 so G runs 1..4, w0=1024), one call, against one
+    # jetlong_prefill per sequence on the same inputs; outside the timed region
+    vl_lens = [int(x) for x in np.random.default_rng(6000).integers(512, 8193, size=64)]
+    vl_max = max(vl_lens)
+    gen = torch.Generator(device=dev).manual_seed(6001)
+    vq = torch.randn((64, 32, vl_max, 128), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vk = torch.randn((64, 8, vl_max, 128), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vv = torch.randn((64, 8, vl_max, 128), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vo = torch.empty_like(vq)
+    vl_kw = dict(w0=1024, w_pretrained=2048, rope_theta=1e6, scale=1.0 / math.sqrt(128), stream=stream)
+
+    def varlen_call():
+        jl.prefill_varlen(vq, vk, vv, vl_lens, vo, **vl_kw)
+
+    per_seq = [(vq[b:b + 1, :, :n].contiguous(), vk[b:b + 1, :, :n].contiguous(),
+                vv[b:b + 1, :, :n].contiguous()) for b, n in enumerate(vl_lens)]
+
+    def per_seq_call():
+        for sq_, sk_, sv_ in per_seq:
+            jl.prefill(sq_, sk_, sv_, **vl_kw)
+
+    vl_res = {}
+    for name, fn in (("one_call", varlen_call), ("one_prefill_per_sequence", per_seq_call)):
+        fn()
+        l0 = jl.launch_count()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        vl_res[name] = (max_over_ranks(a.elapsed_time(b_)), jl.launch_count() - l0)
+    jl.device_status(stream)
+    vl_flops = sum(prefill_flops(I.C4.with_(B=1, L=n, w_pretrained=2048, w0=1024))[1] for n in vl_lens)
+    del vq, vk, vv, vo, per_seq
+
     # ---------------- decode over a standard RoPE cache (jetlong_decode_rope_cache),
     # one pass of the same 64 steps outside the timed region; the kernel's work
     # does not depend on the cached values, so the resident cache bytes serve
@@ -837,6 +874,19 @@ def main():
                             "tflops_computed": round(whole_job_rate(plain_computed, world, plain_ms * 1e-3) / 1e12, 2),
                             "bifocal_over_plain_time": round(pre_ms / plain_ms, 4)}},
             "other_prefill_configs": other,
+            "varlen_batch": {
+                "sequences": 64, "lengths": "seeded uniform in [512, 8192]", "tokens": int(sum(vl_lens)),
+                "Hq": 32, "Hkv": 8, "d": 128, "w_pretrained": 2048, "w0": 1024,
+                "flops_computed": vl_flops,
+                "one_call": {"ms": round(vl_res["one_call"][0], 3), "launches": vl_res["one_call"][1],
+                             "tflops_computed": round(world * vl_flops / (vl_res["one_call"][0] * 1e-3) / 1e12, 2),
+                             "frac_of_burst_bf16": round(vl_flops / (vl_res["one_call"][0] * 1e-3) / 1e12
+                                                         / peaks["bf16_tflops"], 4)},
+                "one_prefill_per_sequence": {
+                    "ms": round(vl_res["one_prefill_per_sequence"][0], 3),
+                    "launches": vl_res["one_prefill_per_sequence"][1],
+                    "tflops_computed": round(world * vl_flops / (vl_res["one_prefill_per_sequence"][0] * 1e-3) / 1e12,
+                                             2)}},
             "decode": {"ms_per_token_step": round(dec_ms / wd.steps, 4),
                        "gbs_kv": round(dec_gbs, 1), "bytes_per_pass_kv": kv_bytes,
                        "bytes_per_pass_all": all_bytes, "tokens_per_s": round(dec_tok_s, 1),

@@ -116,7 +116,10 @@ int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache,
  *   lse (optional, may be NULL): float [B,Hq,Lmax] device array, 4-byte
  *   aligned; row i of sequence b receives log sum_j exp(scale * logit_ij)
  *   (natural log; the statistic an LSE merge of partial attentions needs).
- * Other arguments and errors as jetlong_prefill; one launch per sequence. */
+ * Other arguments and errors as jetlong_prefill.  bf16: one prefill launch
+ * (after a range scan) per 64 sequences, its grid over the query blocks of all
+ * of them, heaviest first; padding rows of q and k may hold anything.  fp32:
+ * one launch per sequence. */
 int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                            int B, int Hq, int Hkv, const int32_t* lens, int Lmax, int d,
                            int w0, int w_pretrained, double rope_theta, float scale,

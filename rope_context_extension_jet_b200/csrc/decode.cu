@@ -490,6 +490,9 @@ __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int 
                                              float& ka, float& kc)
 {
     const int t = lane & 3;
+    // two independent accumulators (first / second halves of the pairs), summed
+    // at the end: half the dependent chain of MMAs
+    float c2[4] = {0.f, 0.f, 0.f, 0.f};
     c[0] = c[1] = c[2] = c[3] = 0.f;
     // ldmatrix.x4 rows: lanes 0-7 keys 0-7 / chunk lo, 8-15 keys 8-15 / lo, 16-23 keys 0-7 / hi, 24-31 keys 8-15 / hi
     const int lkey = kw + (lane & 7) + ((lane >> 3) & 1) * 8, lhalf = lane >> 4;
@@ -548,8 +551,10 @@ __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int 
             hi[kb][r] = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
         }
         mma_f16(c, lo[kb], qb[kb][0], qb[kb][1]);
-        mma_f16(c, hi[kb], qb[kb + D / 32][0], qb[kb + D / 32][1]);
+        mma_f16(c2, hi[kb], qb[kb + D / 32][0], qb[kb + D / 32][1]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] += c2[i];
 }
 
 template <int D, int HPB>

@@ -172,10 +172,13 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
     return ok();
 }
 
+// vl_n > 0 (bf16 only): a variable-length batch of vl_n <= 64 sequences with
+// lengths vl_lens[0..vl_n) in planes of Lcap = Cst = C rows, P = 0, in one launch.
 static int prefill_entry(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                          int Hq, int Hkv, int P, int C, int Cst, int Lcap, int d, int w0,
                          int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
-                         void* stream, int window_rot = -1, int g_len = 0)
+                         void* stream, int window_rot = -1, int g_len = 0, int vl_n = 0,
+                         const int32_t* vl_lens = nullptr)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -203,13 +206,25 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     jl::make_rope_turns(&p.turns, d, rope_theta);
     p.dev_error = derr;
+    jl::ScanRows rows{};
+    if (vl_n > 0) {
+        p.vl_n = vl_n;
+        rows.n = vl_n;
+        rows.hq = Hq;
+        rows.hkv = Hkv;
+        for (int b = 0; b < vl_n; ++b) {
+            p.vl_len[b] = rows.len[b] = vl_lens[b];
+            p.vl_G[b] = (int)jetlong_group_size(vl_lens[b], w_pretrained);
+        }
+    }
     int n = 0;
     if (dtype == JETLONG_BF16) {
         // largest |q| and |k| of the rows this call uses, for the power-of-two
         // operand scales of the fp16 Q K^T (see range_scan.cu)
         uint32_t* slot = next_range_slot(&e);
         if (!slot) return fail(JETLONG_ERR_CUDA, "range slots: %s", cudaGetErrorString(e));
-        e = jl::launch_range_scan(q, C, Cst, B * Hq, k, L, Lcap, B * Hkv, d, slot, (cudaStream_t)stream, &n);
+        e = jl::launch_range_scan(q, C, Cst, B * Hq, k, L, Lcap, B * Hkv, d, slot, (cudaStream_t)stream, &n,
+                                  vl_n > 0 ? &rows : nullptr);
         g_launches += n;
         n = 0;
         if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "range scan launch: %s", cudaGetErrorString(e));
@@ -254,13 +269,24 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3))
         return fail(JETLONG_ERR_INVALID_ARG, "lse must be 4-byte aligned");
     const size_t el = dtype == JETLONG_FP32 ? 4 : 2;
-    for (int b = 0; b < B; ++b) {
-        // sequence b: its own planes, its own length and G, one launch
-        const size_t qo = (size_t)b * Hq * Lmax * d * el, ko = (size_t)b * Hkv * Lmax * d * el;
-        int st = prefill_entry(static_cast<const char*>(q) + qo, static_cast<const char*>(k) + ko,
+    // bf16: up to 64 sequences per launch (one grid over their query blocks,
+    // heaviest first, each with its own length and G); fp32: one launch per
+    // sequence
+    const int per = dtype == JETLONG_BF16 ? 64 : 1;
+    for (int b0 = 0; b0 < B; b0 += per) {
+        const int nb = B - b0 < per ? B - b0 : per;
+        const size_t qo = (size_t)b0 * Hq * Lmax * d * el, ko = (size_t)b0 * Hkv * Lmax * d * el;
+        int st;
+        if (per == 1)
+            st = prefill_entry(static_cast<const char*>(q) + qo, static_cast<const char*>(k) + ko,
                                static_cast<const char*>(v) + ko, static_cast<char*>(out) + qo,
-                               lse ? lse + (size_t)b * Hq * Lmax : nullptr, 1, Hq, Hkv, 0, lens[b], Lmax,
+                               lse ? lse + (size_t)b0 * Hq * Lmax : nullptr, 1, Hq, Hkv, 0, lens[b0], Lmax,
                                Lmax, d, w0, w_pretrained, rope_theta, scale, dtype, stream);
+        else
+            st = prefill_entry(static_cast<const char*>(q) + qo, static_cast<const char*>(k) + ko,
+                               static_cast<const char*>(v) + ko, static_cast<char*>(out) + qo,
+                               lse ? lse + (size_t)b0 * Hq * Lmax : nullptr, nb, Hq, Hkv, 0, Lmax, Lmax, Lmax, d,
+                               w0, w_pretrained, rope_theta, scale, dtype, stream, -1, 0, nb, lens + b0);
         if (st != JETLONG_OK) return st;
     }
     return ok();

@@ -110,6 +110,12 @@ struct PrefillProblem {
     // bf16: two words (largest |q|, largest |k| as bf16 magnitude bits) written
     // by launch_range_scan on the same stream before the prefill kernel
     const uint32_t* range;
+    // bf16 variable-length batch in one launch (vl_n > 0, at most 64
+    // sequences): lengths and group sizes of sequences 0..vl_n-1; B = vl_n, P = 0,
+    // q / out / k / v planes of Cst = Lcap = L = the longest length (L, C are
+    // then the batch maximum)
+    int vl_n;
+    int vl_len[64], vl_G[64];
 };
 
 struct DecodeProblem {
@@ -159,7 +165,14 @@ cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStr
 // Largest magnitude of the used rows of q (planes of Cst rows, rows [0, C)) and
 // of k (planes of Lcap rows, rows [0, L)), bf16, as 15-bit magnitude bits into
 // range[0] and range[1] (zeroed first on the stream).
+// rows (optional): per-sequence row counts of a variable-length batch, plane pl
+// of q (k) belonging to sequence pl / hq (pl / hkv).
+struct ScanRows {
+    int n, hq, hkv;
+    int len[64];
+};
 cudaError_t launch_range_scan(const void* q, int C, int Cst, int q_planes, const void* k, int L, int Lcap,
-                              int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch);
+                              int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch,
+                              const ScanRows* rows = nullptr);
 
 }  // namespace jl

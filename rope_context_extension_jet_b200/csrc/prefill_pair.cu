@@ -81,10 +81,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const int qb = p.nqb - 1 - (int)(blockIdx.x >> 1);  // heaviest query blocks first
+    // the pair's sequence and query block (heaviest query blocks first); a
+    // unit past the end of a shorter sequence of a variable-length batch has no
+    // work (both CTAs of the pair see the same unit)
+    SeqView sv;
+    if (!seq_view(p, (int)(blockIdx.x >> 1), (int)blockIdx.z, sv)) return;
+    const int qb = sv.qb, b = sv.b;
     const int hq4 = blockIdx.y * 4;                      // first of the pair's four query heads
     const int h0 = hq4 + 2 * (int)rank;                  // this CTA's two heads
-    const int b = blockIdx.z;
     const int kvh = hq4 / (p.Hq / p.Hkv);
     // barriers of CTA 0, as cluster addresses (both CTAs arrive on them)
     const uint32_t lbar = mapa_shared(smem_u32(bars), 0);
@@ -111,7 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars[P_DRAIN], 1);
         *abort_flag = 0;
-        *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
+        *plan = plan_tiles(p.P + qb * BM, sv.L, sv.w0);
         if (p.window_rot >= 0) plan->nR = 0;  // windowed pass: the local tiles only
         // after a bounded wait expired anywhere in the grid (error word set),
         // later pairs skip their work; CTA 0 decides for both
@@ -259,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (ok) {
             for (int h = 0; h < 2; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                    rotate_tile<D, BM, true, true>(smem + h * S::QTILE, t, p, [&](int r) { return div_g(i0 + r, sv); }, stc,
                                              sts, lq);
                 else
                     rotate_tile<D, BM, true, true>(smem + h * S::QTILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
@@ -276,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 if (!warp_wait<true>(&bars[P_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x432)) { ok = false; break; }
                 for (int h = 0; h < 2; ++h)
                     rotate_tile<D, BM, false, true>(smem + h * S::QTILE, t, p,
-                                              [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
+                                              [&](int r) { return i0 + r - div_g(i0 + r, sv); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(lead(P_QREADY1));
@@ -285,7 +289,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
             unsigned char* kt = smem + S::K0 + s * S::KTILE;
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return div_g(j0 + r, p); }, stc, sts, lk);
+                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return div_g(j0 + r, sv); }, stc, sts, lk);
             else
                 rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
             fence_proxy_async_smem();
@@ -300,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int hh = (warp - 8) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         const uint32_t pfull = lead(P_PFULL + 2 * hh);
-        softmax_role<D, true>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128, lane_base + 256 + hh * 128,
+        softmax_role<D, true>(p, sv, tp, h0 + hh, tid & 127, lane_base + hh * 128, lane_base + 256 + hh * 128,
                               &bars[P_SFULL + hh], &bars[P_PVDONE + hh],
                               [pfull](int half) { mbar_arrive_cluster(pfull + 8u * (uint32_t)half); }, abort_flag);
     }
@@ -327,7 +331,8 @@ cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
     if ((e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
         return e;
-    dim3 grid(2 * p.nqb, pp.Hq / 4, pp.B);
+    // variable-length: x over (query-block level, sequence), one z
+    dim3 grid(p.vl_n ? 2 * p.vl_nqb_max * p.vl_n : 2 * p.nqb, pp.Hq / 4, p.vl_n ? 1 : pp.B);
     prefill_pair_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }

@@ -40,6 +40,8 @@
 // Every mbarrier wait is bounded; on expiry the CTA records an error code in
 // the library's device error word, stops, drains its own copies and MMAs with
 // bounded waits, frees TMEM and returns.
+#include <algorithm>
+
 #include "prefill_tc_common.cuh"
 
 namespace jl {
@@ -82,8 +84,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     TilePlan* plan = reinterpret_cast<TilePlan*>(tmem_slot + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qb = p.nqb - 1 - (int)blockIdx.x;  // heaviest query blocks first
-    const int h0 = blockIdx.y * NH, b = blockIdx.z;
+    // the CTA's sequence and query block (heaviest query blocks first); a unit
+    // past the end of a shorter sequence of a variable-length batch has no work
+    SeqView sv;
+    if (!seq_view(p, (int)blockIdx.x, (int)blockIdx.z, sv)) return;
+    const int qb = sv.qb, b = sv.b;
+    const int h0 = blockIdx.y * NH;
     const int kvh = h0 / (p.Hq / p.Hkv);
 
     // after a bounded wait expired anywhere in the grid (error word set), later
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
-        *plan = plan_tiles(p.P + qb * BM, p.L, p.w0);
+        *plan = plan_tiles(p.P + qb * BM, sv.L, sv.w0);
         if (p.window_rot >= 0) plan->nR = 0;  // windowed pass: the local tiles only
         fence_mbar_init();
     }
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok) {
             for (int h = 0; h < NH; ++h) {
                 if (nR > 0 || p.window_rot == 1)
-                    rotate_tile<D, BM, true, false>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, p); }, stc,
+                    rotate_tile<D, BM, true, false>(smem + h * S::TILE, t, p, [&](int r) { return div_g(i0 + r, sv); }, stc,
                                              sts, lq);
                 else
                     rotate_tile<D, BM, true, false>(smem + h * S::TILE, t, p, [&](int r) { return i0 + r; }, stc, sts, lq);
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!warp_wait(&bars[B_QFREE], 0, abort_flag, p.dev_error, p.wait_cycles, 0x322)) { ok = false; break; }
                 for (int h = 0; h < NH; ++h)
                     rotate_tile<D, BM, false, false>(smem + h * S::TILE, t, p,
-                                          [&](int r) { return i0 + r - div_g(i0 + r, p); }, stc, sts, 1.f);
+                                          [&](int r) { return i0 + r - div_g(i0 + r, sv); }, stc, sts, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_QREADY1]);
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x323)) { ok = false; break; }
             const uint32_t j0 = (uint32_t)(kb * BN);
             if (e < nR || p.window_rot == 1)
-                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, p); }, stc,
+                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, sv); }, stc,
                                          sts, lk);
             else
                 rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
@@ -293,7 +299,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (hh < NH) {
             const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
             uint64_t* pfull = &bars[B_PFULL + 2 * hh];
-            softmax_role<D, false>(p, tp, qb, h0 + hh, b, tid & 127, lane_base + hh * 128,
+            softmax_role<D, false>(p, sv, tp, h0 + hh, tid & 127, lane_base + hh * 128,
                                    lane_base + 256 + hh * 128, &bars[B_SFULL + hh], &bars[B_PVDONE + hh],
                                    [pfull](int half) { mbar_arrive(pfull + half); }, abort_flag);
         }
@@ -321,7 +327,8 @@ cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
     constexpr int smem = TcSmem<D, NH>::TOTAL;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
         return e;
-    dim3 grid(p.nqb, pp.Hq / NH, pp.B);
+    // variable-length: x over (query-block level, sequence), one z
+    dim3 grid(p.vl_n ? p.vl_nqb_max * p.vl_n : p.nqb, pp.Hq / NH, p.vl_n ? 1 : pp.B);
     kern<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
@@ -390,6 +397,13 @@ TcParams make_params(const PrefillProblem& pp)
     p.wait_cycles = pp.wait_cycles > 0 ? pp.wait_cycles : kPrefillWaitCycles;
     p.inject = pp.inject;
     p.range = pp.range;
+    p.vl_n = pp.vl_n;
+    p.vl_nqb_max = 0;
+    for (int b = 0; b < pp.vl_n; ++b) {
+        p.vl_len[b] = pp.vl_len[b];
+        p.vl_nqb_max = std::max(p.vl_nqb_max, (pp.vl_len[b] + BM - 1) / BM);
+        make_div_magic((uint32_t)pp.vl_G[b], &p.vl_div[b][0], &p.vl_div[b][1], &p.vl_div[b][2]);
+    }
     return p;
 }
 

@@ -22,6 +22,7 @@ namespace jl {
 namespace tc {
 
 constexpr int BM = 128, BN = 128;
+constexpr int kVarlenMax = 64;  // sequences of one variable-length launch
 constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
@@ -44,7 +45,47 @@ struct TcParams {
     // largest |q| and |k| of this call as bf16 magnitude bits, written by the
     // range scan launched just before on the same stream
     const uint32_t* range;
+    // variable-length batches (vl_n > 0): sequence b of the launch has length
+    // vl_len[b] (rows [0, vl_len[b]) of planes of Cst rows), its own G and
+    // floor(x / G) constants; the grid's x runs over (query-block level, b)
+    int vl_n, vl_nqb_max;
+    int vl_len[kVarlenMax];
+    uint32_t vl_div[kVarlenMax][3];
 };
+
+// The sequence and query block a CTA (pair) works on, with that sequence's
+// length, window and floor(x / G) constants.
+struct SeqView {
+    int b, qb, L, w0;
+    uint32_t div_m, div_s1, div_s2;
+};
+
+// Work unit `unit` (the CTA's place along the grid's x, heaviest first) of the
+// launch, batch index bz (blockIdx.z).  Returns false for a unit past the end
+// of a shorter sequence of a variable-length batch (the CTA then has no work).
+__device__ __forceinline__ bool seq_view(const TcParams& p, int unit, int bz, SeqView& v)
+{
+    if (p.vl_n == 0) {
+        v.b = bz;
+        v.qb = p.nqb - 1 - unit;
+        v.L = p.L;
+        v.w0 = p.w0;
+        v.div_m = p.div_m;
+        v.div_s1 = p.div_s1;
+        v.div_s2 = p.div_s2;
+        return true;
+    }
+    // all sequences' blocks of one level (counted from the longest sequence's
+    // last block) before the next lighter level
+    v.b = unit % p.vl_n;
+    v.qb = p.vl_nqb_max - 1 - unit / p.vl_n;
+    v.L = p.vl_len[v.b];
+    v.w0 = min(p.w0, v.L);
+    v.div_m = p.vl_div[v.b][0];
+    v.div_s1 = p.vl_div[v.b][1];
+    v.div_s2 = p.vl_div[v.b][2];
+    return v.qb * BM < v.L;
+}
 
 // ------------------------------------------------------------ operand range
 // The Q K^T operands are rounded to fp16 (an 11-bit significand: the inputs'
@@ -77,12 +118,12 @@ __device__ __forceinline__ uint32_t ld_range(const uint32_t* p)
     return v;
 }
 
-__device__ __forceinline__ uint32_t div_g(uint32_t n, const TcParams& p)
+__device__ __forceinline__ uint32_t div_g(uint32_t n, const SeqView& v)
 {
     // Granlund & Montgomery, "Division by Invariant Integers using
     // Multiplication" (1994), Fig. 4.1: exact for all 32-bit n.
-    const uint32_t t1 = __umulhi(p.div_m, n);
-    return (t1 + ((n - t1) >> p.div_s1)) >> p.div_s2;
+    const uint32_t t1 = __umulhi(v.div_m, n);
+    return (t1 + ((n - t1) >> v.div_s1)) >> v.div_s2;
 }
 
 // Class of the tile (query rows from position i_lo, key block kb): every pair
@@ -279,13 +320,13 @@ __device__ __forceinline__ void rope_steps(int t, const TcParams& p, float2 (&st
 // (`arrive_p(half)`); finally O / l -> out.
 // s_col / o_col are this warp's TMEM addresses of S and O.
 template <int D, bool CLUSTER, class ArriveP>
-__device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& tp, int qb, int head, int b,
+__device__ __forceinline__ void softmax_role(const TcParams& p, const SeqView& sv, const TilePlan& tp, int head,
                                              int r, uint32_t s_col, uint32_t o_col, uint64_t* sfull,
                                              uint64_t* pvdone, ArriveP arrive_p, volatile int* abort_flag)
 {
     const int lane = r & 31;
-    const int L = p.L;
-    const int i_lo = p.P + qb * BM;
+    const int L = sv.L, b = sv.b;
+    const int i_lo = p.P + sv.qb * BM;
     const int i = i_lo + r;
     const int NE = tp.count();
     // scale * log2(e), times 2^-(e_q + e_k) to undo the operand scales; kept in
@@ -298,7 +339,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
     for (int e = 0; e < NE; ++e) {
         const int kb = tp.kb(e);
         const bool phase_r = e < tp.nR;
-        const int cls = tile_class(i_lo, kb, L, p.w0);
+        const int cls = tile_class(i_lo, kb, L, sv.w0);
         if (!warp_wait<CLUSTER>(sfull, e & 1, abort_flag, p.dev_error, p.wait_cycles, 0x331)) { ok = false; break; }
         tc_fence_after();
         float x[BN];
@@ -320,7 +361,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const TilePlan& 
         const int j0 = kb * BN;
         const bool need_mask = (j0 + BN - 1 > i_lo) || (j0 + BN > L) || cls == CLS_BAND;
         if (need_mask) {
-            const int dw = i - j0 - p.w0;  // pair (i, j0 + u) is local iff u > dw
+            const int dw = i - j0 - sv.w0;  // pair (i, j0 + u) is local iff u > dw
 #pragma unroll
             for (int u = 0; u < BN; ++u) {
                 const int j = j0 + u;

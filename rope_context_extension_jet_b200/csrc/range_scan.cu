@@ -20,17 +20,22 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
     return r;
 }
 
-// grid: (blocks per plane, planes (strided), 2 tensors); 256 threads
+// grid: (blocks per plane, planes (strided), 2 tensors); 256 threads.  With
+// rows.n > 0, plane pl of q (k) belongs to sequence pl / rows.hq (pl / rows.hkv)
+// and only its rows [0, rows.len[that sequence]) are read.
 __global__ void __launch_bounds__(256) range_scan_kernel(const uint4* q, long long q_vecs, long long q_stride,
                                                          int q_planes, const uint4* k, long long k_vecs,
-                                                         long long k_stride, int k_planes, uint32_t* range)
+                                                         long long k_stride, int k_planes, int vpr,
+                                                         const ScanRows rows, uint32_t* range)
 {
     const bool is_k = blockIdx.z == 1;
     const uint4* base = is_k ? k : q;
-    const long long nv = is_k ? k_vecs : q_vecs, stride = is_k ? k_stride : q_stride;
+    const long long stride = is_k ? k_stride : q_stride;
     const int planes = is_k ? k_planes : q_planes;
     uint32_t acc = 0u;
     for (int pl = blockIdx.y; pl < planes; pl += gridDim.y) {
+        const long long nv = rows.n ? (long long)rows.len[pl / (is_k ? rows.hkv : rows.hq)] * vpr
+                                    : (is_k ? k_vecs : q_vecs);
         const uint4* row = base + (long long)pl * stride;
         for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < nv;
              v += (long long)gridDim.x * blockDim.x) {
@@ -53,7 +58,8 @@ __global__ void __launch_bounds__(256) range_scan_kernel(const uint4* q, long lo
 }  // namespace
 
 cudaError_t launch_range_scan(const void* q, int C, int Cst, int q_planes, const void* k, int L, int Lcap,
-                              int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch)
+                              int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch,
+                              const ScanRows* rows)
 {
     cudaError_t e = cudaMemsetAsync(range, 0, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
@@ -70,9 +76,11 @@ cudaError_t launch_range_scan(const void* q, int C, int Cst, int q_planes, const
     if (bx > cap) bx = cap;
     if (bx < 1) bx = 1;
     dim3 grid((unsigned)bx, (unsigned)by, 2);
+    ScanRows r{};
+    if (rows) r = *rows;
     range_scan_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(q), q_vecs, (long long)Cst * vpr, q_planes,
                                            static_cast<const uint4*>(k), k_vecs, (long long)Lcap * vpr, k_planes,
-                                           range);
+                                           (int)vpr, r, range);
     e = cudaGetLastError();
     if (e == cudaSuccess) *nlaunch += 1;
     return e;

@@ -256,16 +256,23 @@ def test_chunk_of_128k_sequence_sampled():
 # 1e-4 for fp32.
 
 def varlen_case(name, lens, *, dtype="bf16", Hq=4, Hkv=1, d=128, w_pre=100, w0=17, theta=1e6,
-                index=70, pad=5):
+                index=70, pad=5, nan_qk_padding=False, launches=None):
     import torch
     B, Lmax = len(lens), max(lens) + pad
     w = I.PrefillWorkload(name, index, dtype, B, Hq, Hkv, d, Lmax, w_pre, w0, theta)
     q, k, v = I.prefill_inputs(w)
-    qd = to_device(q)
+    qd, kd = to_device(q), to_device(k)
+    if nan_qk_padding:  # padding rows of q and k may hold anything (those of v must be finite)
+        for b, Lb in enumerate(lens):
+            qd[b, :, Lb:] = float("nan")
+            kd[b, :, Lb:] = float("nan")
     out = torch.full_like(qd, float("nan"))
-    out, lse = jl.prefill_varlen(qd, to_device(k), to_device(v), lens, out, w0=w0, w_pretrained=w_pre,
+    before = jl.launch_count()
+    out, lse = jl.prefill_varlen(qd, kd, to_device(v), lens, out, w0=w0, w_pretrained=w_pre,
                                  rope_theta=theta, scale=w.scale, with_lse=True)
     jl.device_status()
+    if launches is not None:
+        assert jl.launch_count() - before == launches
     got, got_lse = to_host_f64(out), lse.double().cpu().numpy()
     tol = 2e-2 if dtype == "bf16" else 1e-4
     for b, Lb in enumerate(lens):
@@ -293,6 +300,18 @@ def test_varlen_fp32(d):
 def test_varlen_lengths_cross_group_sizes():
     # w_pretrained = 256: G = 1, 2, 4, 5 for the four sequences
     varlen_case("varlen-G", [256, 257, 1024, 1025], Hq=8, Hkv=2, w_pre=256, w0=100, index=73)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 2), (2, 2)])
+def test_varlen_one_launch_for_64_sequences(Hq, Hkv):
+    # bf16: one range scan + one prefill launch per 64 sequences (70 here: two
+    # of each), every sequence with its own length and G; NaN in the padding
+    # rows of q and k must not reach any output
+    rng = np.random.default_rng(74)
+    lens = [int(x) for x in rng.integers(1, 300, size=70)]
+    lens[3], lens[40] = 300, 129
+    varlen_case("varlen-70", lens, Hq=Hq, Hkv=Hkv, w_pre=64, w0=40, index=74, nan_qk_padding=True,
+                launches=4)
 
 
 # ---------------------------------------------------------------- inclusion-exclusion form
