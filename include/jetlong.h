@@ -133,8 +133,10 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
  * The result equals jetlong_prefill's up to rounding; it exists to compare
  * the two forms.  Arguments as jetlong_prefill, plus a device workspace of at
  * least jetlong_prefill_ie_workspace_size(B, Hq, L, d, dtype) bytes (16-byte
- * aligned, caller-owned; the three pass outputs and their LSEs).  Four
- * launches; when w0 = 0, pass B alone and a device-to-device copy into out. */
+ * aligned, caller-owned; the three pass outputs in fp32 -- the merge subtracts
+ * nearly equal terms, so they are not rounded to bf16 first -- and their
+ * LSEs).  Three passes (each a range scan and a prefill launch for bf16) and
+ * the merge; when w0 = 0, pass B alone, written into out. */
 size_t jetlong_prefill_ie_workspace_size(int B, int Hq, int L, int d, jetlong_dtype dtype);
 int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
                        int B, int Hq, int Hkv, int L, int d,
@@ -260,6 +262,26 @@ int jetlong_selftest_wait_timeout(void* stream);
 #define JETLONG_INJECT_PREFILL_KEY_TILE 1
 #define JETLONG_INJECT_DECODE_COPY 2
 int jetlong_debug_inject_timeout(int site, long long wait_cycles);
+
+/* Test hooks (the pages have no counterpart): the device helpers of the
+ * attention kernels on their own, for checks against host computations.
+ *
+ * jetlong_debug_rope_phase: d_out[2 (i d/2 + m) + {0, 1}] = (cos, sin) of
+ * d_pos[i] * theta_m, theta_m = rope_theta^(-2m/d), m < d/2, as the kernels
+ * form it (exact fixed-point turn fraction, then sincospif when `accurate`,
+ * else __sincosf).  d_pos: n uint32 positions; d_out: 2 n d/2 floats (device).
+ *
+ * jetlong_debug_tile_plan: for the query blocks qb (128 rows each) of rows
+ * [P, P + C) against keys [0, L = P + C) with window w0: d_plan[3 qb + {0,1,2}]
+ * = (nR, kE0, nkb) -- the remote-phase tiles are key blocks [0, nR), the
+ * exact-phase tiles [kE0, nkb) -- and d_cls[qb max_kb + kb] (kb < min(nkb,
+ * max_kb)) the class of tile (qb, kb): 0 every causal pair remote, 1 every pair
+ * local, 2 both.  Device arrays of 3 ceil(C / 128) int32 and ceil(C / 128)
+ * max_kb int8.  Both return JETLONG_OK, JETLONG_ERR_INVALID_ARG or
+ * JETLONG_ERR_CUDA; asynchronous on stream. */
+int jetlong_debug_rope_phase(const uint32_t* d_pos, int64_t n, int d, double rope_theta, int accurate,
+                             float* d_out, void* stream);
+int jetlong_debug_tile_plan(int P, int C, int w0, int max_kb, int32_t* d_plan, int8_t* d_cls, void* stream);
 
 /* Message for the last failing call on this host thread ("" if none). */
 const char* jetlong_last_error(void);

@@ -24,7 +24,7 @@ __all__ = [
     "prefill_chunk", "prefill_varlen", "prefill_ie", "prefill_streamed", "decode_workspace_size",
     "decode", "decode_rope_cache", "decode_noalloc", "device_status", "last_error", "launch_count",
     "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout", "debug_inject_timeout",
-    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY",
+    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY", "debug_rope_phase", "debug_tile_plan",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +91,10 @@ def load_library(path: str | None = None):
         lib.jetlong_selftest_wait_timeout.argtypes = [vp]
         lib.jetlong_debug_inject_timeout.restype = i32
         lib.jetlong_debug_inject_timeout.argtypes = [i32, ctypes.c_longlong]
+        lib.jetlong_debug_rope_phase.restype = i32
+        lib.jetlong_debug_rope_phase.argtypes = [vp, i64, i32, dbl, i32, vp, vp]
+        lib.jetlong_debug_tile_plan.restype = i32
+        lib.jetlong_debug_tile_plan.argtypes = [i32, i32, i32, i32, vp, vp, vp]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -399,6 +403,34 @@ def debug_inject_timeout(site: int, wait_cycles: int):
     device_status() raises TIMEOUT (jetlong_debug_inject_timeout)."""
     lib = load_library()
     _check(lib.jetlong_debug_inject_timeout(int(site), int(wait_cycles)), lib)
+
+
+def debug_rope_phase(pos, d: int, rope_theta: float, accurate: bool, stream=None):
+    """(cos, sin) of pos[i] * theta_m as the kernels form them: float32 CUDA
+    tensor [n, d/2, 2] (test hook jetlong_debug_rope_phase).  pos: int32 CUDA
+    tensor holding uint32 positions."""
+    import torch
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32 (uint32 bit patterns)")
+    out = torch.empty((pos.numel(), d // 2, 2), dtype=torch.float32, device=pos.device)
+    lib = load_library()
+    _check(lib.jetlong_debug_rope_phase(_dev(pos, "pos"), pos.numel(), int(d), float(rope_theta),
+                                        1 if accurate else 0, _dev(out, "out"), _stream(stream)), lib)
+    return out
+
+
+def debug_tile_plan(P: int, C: int, w0: int, max_kb: int, stream=None):
+    """The prefill's tile plan (nR, kE0, nkb) per query block and the class of
+    every tile (0 remote, 1 local, 2 both; -1 past nkb): test hook
+    jetlong_debug_tile_plan.  Returns (plan [nqb, 3] int32, cls [nqb, max_kb] int8)."""
+    import torch
+    nqb = (C + 127) // 128
+    plan = torch.empty((nqb, 3), dtype=torch.int32, device="cuda")
+    cls = torch.full((nqb, max_kb), -1, dtype=torch.int8, device="cuda")
+    lib = load_library()
+    _check(lib.jetlong_debug_tile_plan(int(P), int(C), int(w0), int(max_kb), _dev(plan, "plan"), _dev(cls, "cls"),
+                                       _stream(stream)), lib)
+    return plan, cls
 
 
 def device_status(stream=None):

@@ -8,16 +8,18 @@
 //   C = window pairs at the aliased positions,
 // whose softmax denominators e^lA, e^lB, e^lC combine exactly:
 //   out = (e^lA O_A + e^lB O_B - e^lC O_C) / (e^lA + e^lB - e^lC).
-// One warp per row (d / 32 elements per lane, contiguous 16-byte loads for
-// bf16 rows of 128); HBM-bound.  Passes with no pairs (lse = -inf) drop out.
+// One warp per row (d / 32 elements per lane); HBM-bound.  Passes with no pairs
+// (lse = -inf) drop out.
 #include "jl_common.cuh"
 
 namespace jl {
 namespace {
 
+// The pass outputs arrive in fp32 (the subtraction cancels, so their rounding
+// to the output type is left to the merged value); out is T.
 template <typename T>
-__global__ void __launch_bounds__(256) ie_merge_kernel(const T* __restrict__ oa, const T* __restrict__ ob,
-                                                       const T* __restrict__ oc, const float* __restrict__ la,
+__global__ void __launch_bounds__(256) ie_merge_kernel(const float* __restrict__ oa, const float* __restrict__ ob,
+                                                       const float* __restrict__ oc, const float* __restrict__ la,
                                                        const float* __restrict__ lb, const float* __restrict__ lc,
                                                        T* __restrict__ out, long long rows, int d)
 {
@@ -33,9 +35,9 @@ __global__ void __launch_bounds__(256) ie_merge_kernel(const T* __restrict__ oa,
     const size_t base = (size_t)row * d;
     for (int e = lane; e < d; e += 32) {
         float acc = 0.f;
-        if (wa != 0.f) acc += wa * load_elem(oa + base + e);
-        if (wb != 0.f) acc += wb * load_elem(ob + base + e);
-        if (wc != 0.f) acc -= wc * load_elem(oc + base + e);
+        if (wa != 0.f) acc += wa * oa[base + e];
+        if (wb != 0.f) acc += wb * ob[base + e];
+        if (wc != 0.f) acc -= wc * oc[base + e];
         store_elem(out + base + e, acc * inv);
     }
 }
@@ -48,14 +50,14 @@ cudaError_t launch_ie_merge(const void* oa, const void* ob, const void* oc, cons
 {
     if (rows <= 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + 7) / 8);
+    const float* a = static_cast<const float*>(oa);
+    const float* b = static_cast<const float*>(ob);
+    const float* c = static_cast<const float*>(oc);
     if (dt == JETLONG_FP32)
-        ie_merge_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(oa), static_cast<const float*>(ob),
-                                                    static_cast<const float*>(oc), la, lb, lc,
-                                                    static_cast<float*>(out), rows, d);
+        ie_merge_kernel<float><<<grid, 256, 0, s>>>(a, b, c, la, lb, lc, static_cast<float*>(out), rows, d);
     else
-        ie_merge_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(oa), static_cast<const __nv_bfloat16*>(ob),
-            static_cast<const __nv_bfloat16*>(oc), la, lb, lc, static_cast<__nv_bfloat16*>(out), rows, d);
+        ie_merge_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a, b, c, la, lb, lc, static_cast<__nv_bfloat16*>(out),
+                                                            rows, d);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) *nlaunch += 1;
     return e;

@@ -178,7 +178,7 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
                          int Hq, int Hkv, int P, int C, int Cst, int Lcap, int d, int w0,
                          int w_pretrained, double rope_theta, float scale, jetlong_dtype dtype,
                          void* stream, int window_rot = -1, int g_len = 0, int vl_n = 0,
-                         const int32_t* vl_lens = nullptr)
+                         const int32_t* vl_lens = nullptr, bool out_f32 = false)
 {
     if (!q || !k || !v || !out) return fail(JETLONG_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -199,6 +199,7 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
     p.P = P; p.C = C; p.Cst = Cst; p.Lcap = Lcap;
     p.lse = lse;
     p.window_rot = window_rot;
+    p.out_f32 = out_f32 && dtype == JETLONG_BF16;
     p.w0 = w0 > L ? L : w0;  // any w0 >= L makes every causal pair local
     // G from the current length (a chunk's P + C), or from g_len when the chunk
     // is part of one whole-sequence prefill
@@ -292,12 +293,13 @@ int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* ou
     return ok();
 }
 
-// Workspace of the three-pass form: O_A, O_B, O_C in the output dtype, then
-// their per-row LSEs (fp32), each segment 256-byte aligned.
+// Workspace of the three-pass form: O_A, O_B, O_C in fp32 (the merge subtracts
+// nearly equal terms, so the passes are not rounded to bf16 first), then their
+// per-row LSEs (fp32), each segment 256-byte aligned.
 static size_t ie_segments(int B, int Hq, int L, int d, jetlong_dtype dtype, size_t* o_bytes, size_t* l_bytes)
 {
-    const size_t el = dtype == JETLONG_FP32 ? 4 : 2;
-    *o_bytes = (((size_t)B * Hq * L * d * el) + 255) & ~(size_t)255;
+    (void)dtype;
+    *o_bytes = (((size_t)B * Hq * L * d * 4) + 255) & ~(size_t)255;
     *l_bytes = (((size_t)B * Hq * L * 4) + 255) & ~(size_t)255;
     return 3 * (*o_bytes + *l_bytes);
 }
@@ -330,23 +332,23 @@ int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out, i
     float* la = reinterpret_cast<float*>(ws + 3 * ob);
     float* lbuf = reinterpret_cast<float*>(ws + 3 * ob + lb);
     float* lc = reinterpret_cast<float*>(ws + 3 * ob + 2 * lb);
-    // B: every causal pair at the aliased positions (the routed kernel with w0 = 0)
-    st = prefill_entry(q, k, v, obuf, lbuf, B, Hq, Hkv, 0, L, L, L, d, 0, w_pretrained, rope_theta, scale,
-                       dtype, stream);
-    if (st != JETLONG_OK) return st;
     if (w0 == 0) {
-        // no window: the routed output is pass B alone (A and C hold no pairs)
-        cudaError_t e = cudaMemcpyAsync(out, obuf, (size_t)B * Hq * L * d * (dtype == JETLONG_FP32 ? 4 : 2),
-                                        cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
-        if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "copy: %s", cudaGetErrorString(e));
-        return ok();
+        // no window: the routed output is pass B alone (A and C hold no pairs),
+        // written straight into out
+        return prefill_entry(q, k, v, out, nullptr, B, Hq, Hkv, 0, L, L, L, d, 0, w_pretrained, rope_theta, scale,
+                             dtype, stream);
     }
-    // A: window pairs at the exact positions; C: window pairs at the aliased positions
+    // B: every causal pair at the aliased positions (the routed kernel with
+    // w0 = 0); A: window pairs at the exact positions; C: window pairs at the
+    // aliased positions; all three as fp32 rows
+    st = prefill_entry(q, k, v, obuf, lbuf, B, Hq, Hkv, 0, L, L, L, d, 0, w_pretrained, rope_theta, scale,
+                       dtype, stream, -1, 0, 0, nullptr, true);
+    if (st != JETLONG_OK) return st;
     st = prefill_entry(q, k, v, oa, la, B, Hq, Hkv, 0, L, L, L, d, w0, w_pretrained, rope_theta, scale, dtype,
-                       stream, 0);
+                       stream, 0, 0, 0, nullptr, true);
     if (st != JETLONG_OK) return st;
     st = prefill_entry(q, k, v, oc, lc, B, Hq, Hkv, 0, L, L, L, d, w0, w_pretrained, rope_theta, scale, dtype,
-                       stream, 1);
+                       stream, 1, 0, 0, nullptr, true);
     if (st != JETLONG_OK) return st;
     int n = 0;
     cudaError_t e = jl::launch_ie_merge(oa, obuf, oc, la, lbuf, lc, out, (long long)B * Hq * L, d, dtype,
@@ -587,6 +589,34 @@ int jetlong_debug_inject_timeout(int site, long long wait_cycles)
         return fail(JETLONG_ERR_INVALID_ARG, "wait_cycles must be in [1e4, 4e9] (got %lld)", wait_cycles);
     g_inject_site = site;
     g_inject_cycles = wait_cycles;
+    return ok();
+}
+
+int jetlong_debug_rope_phase(const uint32_t* d_pos, int64_t n, int d, double rope_theta, int accurate,
+                             float* d_out, void* stream)
+{
+    if (!d_pos || !d_out) return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (n < 0 || (d != 64 && d != 128) || !(rope_theta > 1.0) || !std::isfinite(rope_theta))
+        return fail(JETLONG_ERR_INVALID_ARG, "need n >= 0, d in {64, 128}, finite rope_theta > 1");
+    jl::RopeTurns turns;
+    jl::make_rope_turns(&turns, d, rope_theta);
+    int nl = 0;
+    cudaError_t e = jl::launch_rope_phase(d_pos, n, d, turns, accurate, d_out, (cudaStream_t)stream, &nl);
+    g_launches += nl;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "rope phase launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int jetlong_debug_tile_plan(int P, int C, int w0, int max_kb, int32_t* d_plan, int8_t* d_cls, void* stream)
+{
+    if (!d_plan || !d_cls) return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (P < 0 || C < 1 || w0 < 0 || max_kb < 1 || (int64_t)P + C > 2147483647LL)
+        return fail(JETLONG_ERR_INVALID_ARG, "need P >= 0, C >= 1, w0 >= 0, max_kb >= 1");
+    const int L = P + C;
+    int nl = 0;
+    cudaError_t e = jl::launch_tile_plan(P, C, L, w0 > L ? L : w0, max_kb, d_plan, d_cls, (cudaStream_t)stream, &nl);
+    g_launches += nl;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "tile plan launch: %s", cudaGetErrorString(e));
     return ok();
 }
 

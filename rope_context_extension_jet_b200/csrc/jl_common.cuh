@@ -116,6 +116,8 @@ struct PrefillProblem {
     // then the batch maximum)
     int vl_n;
     int vl_len[64], vl_G[64];
+    // bf16: write out as fp32 rows (the three-pass form's intermediate passes)
+    int out_f32;
 };
 
 struct DecodeProblem {
@@ -158,6 +160,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int Lcap, int d);
 cudaError_t launch_position_map(int32_t* out, int L, int G, cudaStream_t s, int* nlaunch);
 // Inclusion-exclusion merge of three attention passes (A, B, C) with their
 // per-row LSEs: out = (e^lA O_A + e^lB O_B - e^lC O_C) / (e^lA + e^lB - e^lC).
+// The pass outputs are fp32 rows; out has the element type dt.
 cudaError_t launch_ie_merge(const void* oa, const void* ob, const void* oc, const float* la, const float* lb,
                             const float* lc, void* out, long long rows, int d, jetlong_dtype dt,
                             cudaStream_t s, int* nlaunch);
@@ -165,6 +168,11 @@ cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStr
 // Largest magnitude of the used rows of q (planes of Cst rows, rows [0, C)) and
 // of k (planes of Lcap rows, rows [0, L)), bf16, as 15-bit magnitude bits into
 // range[0] and range[1] (zeroed first on the stream).
+// Test hooks (debug_kernels.cu): the phase helpers and the tile plan on their own.
+cudaError_t launch_rope_phase(const uint32_t* pos, long long n, int d, const RopeTurns& turns, int accurate,
+                              float* out, cudaStream_t s, int* nlaunch);
+cudaError_t launch_tile_plan(int P, int C, int L, int w0, int max_kb, int32_t* plan, int8_t* cls, cudaStream_t s,
+                             int* nlaunch);
 // rows (optional): per-sequence row counts of a variable-length batch, plane pl
 // of q (k) belonging to sequence pl / hq (pl / hkv).
 struct ScanRows {

@@ -390,7 +390,8 @@ TcParams make_params(const PrefillProblem& pp)
     make_div_magic((uint32_t)pp.G, &p.div_m, &p.div_s1, &p.div_s2);
     p.scale_log2 = pp.scale_log2;
     p.turns = pp.turns;
-    p.out = reinterpret_cast<__nv_bfloat16*>(pp.out);
+    p.out = pp.out_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(pp.out);
+    p.out_f32 = pp.out_f32 ? reinterpret_cast<float*>(pp.out) : nullptr;
     p.lse = pp.lse;
     p.window_rot = pp.window_rot;
     p.dev_error = pp.dev_error;

@@ -37,6 +37,7 @@ struct TcParams {
     float scale_log2;
     RopeTurns turns;
     __nv_bfloat16* out;
+    float* out_f32;  // if set, the output rows are written here in fp32 instead of `out`
     float* lse;      // optional
     int window_rot;  // -1 routed; 0 / 1: pairs i - j < w0 only, exact / aliased rotation
     int* dev_error;
@@ -453,7 +454,15 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const SeqView& s
             uint32_t tt[32];
             tmem_ld32(o_col + cc * 32, tt);
             tmem_wait_ld();
-            if (i < L) {
+            if (i < L && p.out_f32) {
+                // fp32 rows (the passes of the three-pass form, merged afterwards)
+                float* frow = p.out_f32 + row * D + cc * 32;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4*>(frow + q * 4) =
+                        make_float4(__uint_as_float(tt[q * 4 + 0]) * inv, __uint_as_float(tt[q * 4 + 1]) * inv,
+                                    __uint_as_float(tt[q * 4 + 2]) * inv, __uint_as_float(tt[q * 4 + 3]) * inv);
+            } else if (i < L) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 v;

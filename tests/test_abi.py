@@ -172,7 +172,9 @@ def test_prefill_varlen_rejects_bad_arguments_on_host(lib, lens, kw, status):
 
 
 def test_prefill_ie_workspace_and_arguments(lib):
-    assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 128, 0) >= 3 * (4 * 600 * 128 * 2 + 4 * 600 * 4)
+    # three fp32 pass outputs and three fp32 LSE arrays, each segment 256-byte aligned
+    assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 128, 0) == 3 * (4 * 600 * 128 * 4 + 9728)
+    assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 128, 1) == 3 * (4 * 600 * 128 * 4 + 9728)
     assert lib.jetlong_prefill_ie_workspace_size(1, 4, 600, 96, 0) == 0
     before = jl.launch_count()
     args = [P, P, P, P, 1, 4, 2, 64, 128, 8, 32, 1e6, 0.088, 0]
