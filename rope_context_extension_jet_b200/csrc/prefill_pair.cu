@@ -43,6 +43,14 @@ constexpr int D = 128;
 constexpr int NS = 5;           // ring depth of the K and V halves
 constexpr int KROWS = BN / 2;   // keys of a K tile held by one CTA
 constexpr int NTHREADS = 512;
+// Registers per thread after setmaxnreg: producer / MMA warpgroup, rotation
+// warpgroup, each of the two softmax warpgroups.  setmaxnreg.inc takes its
+// registers from those the block was launched with (NTHREADS x 128), so the
+// split must not ask for more, or the increase would wait for ever.
+constexpr int kRegsProducer = 56, kRegsRotation = 72, kRegsSoftmax = 192;
+static_assert((kRegsProducer + kRegsRotation + 2 * kRegsSoftmax) * 128 <= NTHREADS * 128,
+              "register split exceeds the launch's registers");
+static_assert(kRegsProducer % 8 == 0 && kRegsRotation % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 
 enum {
     P_QFULL = 0, P_QREADY0, P_QREADY1, P_QFREE,
@@ -139,7 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int nR = tp.nR, NE = tp.count();
 
     if (warp < 4) {
-        regs_dec<56>();
+        regs_dec<kRegsProducer>();
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
@@ -251,7 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
         }
     } else if (warp < 8) {
-        regs_dec<72>();
+        regs_dec<kRegsRotation>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
         float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
@@ -299,7 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (lane == 0 && !(p.inject == kInjectPrefillKeyTile && e == 0)) mbar_arrive_cluster(lead(P_KREADY + s));
         }
     } else {
-        regs_inc<192>();
+        regs_inc<kRegsSoftmax>();
         // -------------------------------------------------------------- softmax (head hh)
         const int hh = (warp - 8) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);

@@ -49,6 +49,14 @@ namespace tc {
 namespace {
 
 constexpr int NSK = 2, NSV = 2, NTHREADS = 512;
+// Registers per thread after setmaxnreg: producer / MMA warpgroup, rotation
+// warpgroup, each of the two softmax warpgroups.  setmaxnreg.inc takes its
+// registers from those the block was launched with (NTHREADS x 128), so the
+// split must not ask for more, or the increase would wait for ever.
+constexpr int kRegsProducer = 56, kRegsRotation = 88, kRegsSoftmax = 184;
+static_assert((kRegsProducer + kRegsRotation + 2 * kRegsSoftmax) * 128 <= NTHREADS * 128,
+              "register split exceeds the launch's registers");
+static_assert(kRegsProducer % 8 == 0 && kRegsRotation % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 
 enum {
     B_QFULL = 0, B_QREADY0, B_QREADY1, B_QFREE,
@@ -134,7 +142,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int nR = tp.nR, NE = tp.count();
 
     if (warp < 4) {
-        regs_dec<56>();
+        regs_dec<kRegsProducer>();
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait(&bars[B_DRAIN], 0);
         }
     } else if (warp < 8) {
-        regs_dec<88>();
+        regs_dec<kRegsRotation>();
         // -------------------------------------------------------------- rotation
         const int t = tid - 128;
         float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
@@ -293,7 +301,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0 && !(p.inject == kInjectPrefillKeyTile && e == 0)) mbar_arrive(&bars[B_KREADY + sk]);
         }
     } else {
-        regs_inc<184>();
+        regs_inc<kRegsSoftmax>();
         // -------------------------------------------------------------- softmax (head hh)
         const int hh = (warp - 8) >> 2;
         if (hh < NH) {
