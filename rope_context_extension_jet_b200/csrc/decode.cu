@@ -31,6 +31,7 @@ constexpr int KROWS = 32;       // key rows per pipeline stage
 constexpr int NCW = 4;          // consumer warps
 constexpr int NT = (NCW + 1) * 32;
 constexpr int kMaxSplits = 256;
+constexpr double kCtaFixedKeys = 256.0;  // per-CTA fixed cost of a decode split, in keys
 
 struct DecodeLaunch {
     int n_splits, chunk, hgroups, hpb;
@@ -401,7 +402,8 @@ struct DecTcCfg {
     static constexpr int PBUF = BIG;                       // [TC_NCW][16 keys][8 heads] bf16
     static constexpr int SQ = PBUF + TC_NCW * 256;         // [2][HPB][D] fp32 rotated queries
     static constexpr int TURNS = SQ + 2 * HPB * D * 4;     // [d/2] uint2 phase constants
-    static constexpr int QEXP = TURNS + (D / 2) * 8;       // [8] int query exponents, [1] large-query flag
+    static constexpr int DELTA = TURNS + (D / 2) * 8;      // [9][d/4] float4 (cos, cos, sin, sin) of 0..8 steps
+    static constexpr int QEXP = DELTA + 9 * (D / 2) * 8;   // [8] int query exponents, [1] large-query flag
     static constexpr int BARS = QEXP + 48;
     static constexpr int END = BARS + 2 * TC_STAGES * 8 + 16;
     static constexpr int TOTAL = END + 1024;
@@ -479,14 +481,41 @@ __device__ __forceinline__ int range_exp_bf16(uint32_t mag)
 
 __device__ __forceinline__ float pow2i_dec(int e) { return __int_as_float((e + 127) << 23); }
 
+// Rotates two adjacent pairs m, m + 1 of one key row: (x, y) of pair m in the
+// low halves of lo / hi, pair m + 1 in the high halves, by the angles with
+// cosines c0, c1 and sines s0, s1 (by minus them for NEG), times lam when
+// SCALED; packs to fp16.
+template <bool SCALED, bool NEG>
+__device__ __forceinline__ void rotate_pairs(uint32_t& lo, uint32_t& hi, float c0, float s0, float c1, float s1,
+                                             float lam)
+{
+    if (SCALED) {
+        c0 *= lam;
+        c1 *= lam;
+        s0 *= lam;
+        s1 *= lam;
+    }
+    if (NEG) {
+        s0 = -s0;
+        s1 = -s1;
+    }
+    const float x0 = bf16_lo(lo), x1 = bf16_hi(lo);
+    const float y0 = bf16_lo(hi), y1 = bf16_hi(hi);
+    lo = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+    hi = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
+}
+
 // S^T for the 16 keys of this warp's block: rotated K fragments times Q^T.
 // Keys of rows g and g + 8 are rotated by the angles of positions pa and pb
-// (by minus those angles when sgn = -1).  SCALED: each key row is first scaled
+// (by minus those angles for NEG); pb - pa must lie in [0, 8], as it does for
+// rows 8 apart.  Row g's angles come from the phase, row g + 8's from them by
+// angle addition with the table of 0..8 steps.  SCALED: each key row is first scaled
 // by its own power of two and ka / kc receive the inverse scales of rows
 // g / g + 8; otherwise the keys are rounded as they are and ka = kc = 1.
-template <int D, bool SCALED>
+template <int D, bool SCALED, bool NEG>
 __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int kw, int lane, uint32_t pa, uint32_t pb,
-                                             float sgn, const uint2* sturns, const uint32_t (&qb)[D / 16][2],
+                                             const uint2* sturns, const float4* sdelta,
+                                             const uint32_t (&qb)[D / 16][2],
                                              float& ka, float& kc)
 {
     const int t = lane & 3;
@@ -526,29 +555,27 @@ __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int 
     ka = pow2i_dec(-ea);
     kc = pow2i_dec(-ec);
     }
+    // row g + 8 sits dpos = pb - pa in [0, 8] positions after row g (exact
+    // positions: 8; grouped positions: the difference of two floor(j / G))
+    const float4* drow = sdelta + min(pb - pa, 8u) * (D / 4);
 #pragma unroll
     for (int kb = 0; kb < D / 32; ++kb) {
-        const int m0 = 16 * kb + 2 * t;
-        // lo[0]: key g, dims m0,m0+1; lo[1]: key g+8; lo[2]: key g, dims m0+8,m0+9; lo[3]: key g+8
+        // lo[kb][2h] / hi[kb][2h]: row g, pairs m, m + 1 (first / second halves
+        // of d); lo[kb][2h + 1] / hi[kb][2h + 1]: row g + 8, same pairs
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const uint32_t pos = (r & 1) ? pb : pa;
-            const float lam = (r & 1) ? lc : la;
-            const int m = m0 + ((r >> 1) ? 8 : 0);
-            const uint2 w0 = sturns[m], w1 = sturns[m + 1];
+        for (int h = 0; h < 2; ++h) {
+            const int m = 16 * kb + 2 * t + 8 * h;
+            const uint4 w = *reinterpret_cast<const uint4*>(sturns + m);  // (hi, lo) of pairs m, m + 1
             float c0, s0, c1, s1;
-            rope_cs_fast(pos, w0.x, w0.y, c0, s0);
-            rope_cs_fast(pos, w1.x, w1.y, c1, s1);
-            if (SCALED) {
-                c0 *= lam;
-                c1 *= lam;
-            }
-            s0 *= SCALED ? sgn * lam : sgn;
-            s1 *= SCALED ? sgn * lam : sgn;
-            const float x0 = bf16_lo(lo[kb][r]), x1 = bf16_hi(lo[kb][r]);
-            const float y0 = bf16_lo(hi[kb][r]), y1 = bf16_hi(hi[kb][r]);
-            lo[kb][r] = pack_f16x2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
-            hi[kb][r] = pack_f16x2(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
+            rope_cs_fast(pa, w.x, w.y, c0, s0);
+            rope_cs_fast(pa, w.z, w.w, c1, s1);
+            // angle addition: (c + i s) of row g times that of dpos steps,
+            // stored as (cos m, cos m+1, sin m, sin m+1)
+            const float4 st = drow[m / 2];
+            const float cb0 = c0 * st.x - s0 * st.z, sb0 = s0 * st.x + c0 * st.z;
+            const float cb1 = c1 * st.y - s1 * st.w, sb1 = s1 * st.y + c1 * st.w;
+            rotate_pairs<SCALED, NEG>(lo[kb][2 * h], hi[kb][2 * h], c0, s0, c1, s1, la);
+            rotate_pairs<SCALED, NEG>(lo[kb][2 * h + 1], hi[kb][2 * h + 1], cb0, sb0, cb1, sb1, lc);
         }
         mma_f16(c, lo[kb], qb[kb][0], qb[kb][1]);
         mma_f16(c2, hi[kb], qb[kb + D / 32][0], qb[kb + D / 32][1]);
@@ -557,7 +584,8 @@ __device__ __forceinline__ void block_logits(float (&c)[4], uint32_t ktile, int 
     for (int i = 0; i < 4; ++i) c[i] += c2[i];
 }
 
-template <int D, int HPB>
+// RC: the cache holds keys already rotated to their own positions (rope_cache).
+template <int D, int HPB, bool RC>
 __global__ void __launch_bounds__(TC_NT, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      DecodeProblem p, DecodeLaunch dl)
@@ -570,6 +598,8 @@ __global__ void __launch_bounds__(TC_NT, 2)
     unsigned char* ring = smem;
     float* sq = reinterpret_cast<float*>(smem + C::SQ);           // [2][HPB][D]
     uint2* sturns = reinterpret_cast<uint2*>(smem + C::TURNS);    // (hi, lo) per frequency
+    float* sdel = reinterpret_cast<float*>(smem + C::DELTA);       // [9][d/4] (cos m, cos m+1, sin m, sin m+1) of 0..8 steps
+    const float4* sdelta = reinterpret_cast<const float4*>(sdel);
     int* qexp = reinterpret_cast<int*>(smem + C::QEXP);            // [HPB] query exponents
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BARS);
     uint64_t* empty = full + TC_STAGES;
@@ -595,6 +625,14 @@ __global__ void __launch_bounds__(TC_NT, 2)
         fence_mbar_init();
     }
     for (int m = tid; m < H; m += TC_NT) sturns[m] = make_uint2(p.turns.hi[m], p.turns.lo[m]);
+    for (int e = tid; e < 9 * H; e += TC_NT) {
+        const int dpos = e / H, m = e % H;
+        float c, sn;
+        rope_cs_accurate((uint32_t)dpos, p.turns.hi[m], p.turns.lo[m], c, sn);
+        float* q4 = sdel + (dpos * (H / 2) + m / 2) * 4 + (m & 1);
+        q4[0] = c;
+        q4[2] = sn;
+    }
     {
         const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0) * D;
         const uint32_t pe = (uint32_t)i, pr = div_g((uint32_t)i, dl);
@@ -717,10 +755,9 @@ __global__ void __launch_bounds__(TC_NT, 2)
             const int ja = jb + g, jc = jb + g + 8;     // the keys of rows g and g + 8
             // raw keys go to j (local) or f(j) (remote); keys stored rotated to
             // j stay (local) or move by f(j) - j <= 0 (remote)
-            const uint32_t ea = p.rope_cache ? 0u : (uint32_t)ja, ec = p.rope_cache ? 0u : (uint32_t)jc;
+            const uint32_t ea = RC ? 0u : (uint32_t)ja, ec = RC ? 0u : (uint32_t)jc;
             const uint32_t fa = div_g((uint32_t)ja, dl), fc = div_g((uint32_t)jc, dl);
-            const uint32_t ra = p.rope_cache ? (uint32_t)ja - fa : fa, rc = p.rope_cache ? (uint32_t)jc - fc : fc;
-            const float rsgn = p.rope_cache ? -1.f : 1.f;
+            const uint32_t ra = RC ? (uint32_t)ja - fa : fa, rc = RC ? (uint32_t)jc - fc : fc;
             // Keys are rounded to fp16 as they are unless that could lose the
             // logits: an element beyond fp16's range (seen as a non-finite
             // logit, as it always is) or a query for which the CTA takes the
@@ -731,13 +768,13 @@ __global__ void __launch_bounds__(TC_NT, 2)
             if (!scaled) {
                 float ka, kc;
                 if (jb >= j_exact) {
-                    block_logits<D, false>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    block_logits<D, false, false>(sc, ktile, kw, lane, ea, ec, sturns, sdelta, qb_ex, ka, kc);
                 } else if (jb + 15 < j_exact) {
-                    block_logits<D, false>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                    block_logits<D, false, RC>(sc, ktile, kw, lane, ra, rc, sturns, sdelta, qb_rm, ka, kc);
                 } else {
                     float se[4];
-                    block_logits<D, false>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
-                    block_logits<D, false>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    block_logits<D, false, RC>(sc, ktile, kw, lane, ra, rc, sturns, sdelta, qb_rm, ka, kc);
+                    block_logits<D, false, false>(se, ktile, kw, lane, ea, ec, sturns, sdelta, qb_ex, ka, kc);
                     if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
                     if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
                 }
@@ -747,13 +784,13 @@ __global__ void __launch_bounds__(TC_NT, 2)
             if (scaled) {
                 float ka, kc;
                 if (jb >= j_exact) {
-                    block_logits<D, true>(sc, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    block_logits<D, true, false>(sc, ktile, kw, lane, ea, ec, sturns, sdelta, qb_ex, ka, kc);
                 } else if (jb + 15 < j_exact) {
-                    block_logits<D, true>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
+                    block_logits<D, true, RC>(sc, ktile, kw, lane, ra, rc, sturns, sdelta, qb_rm, ka, kc);
                 } else {
                     float se[4];
-                    block_logits<D, true>(sc, ktile, kw, lane, ra, rc, rsgn, sturns, qb_rm, ka, kc);
-                    block_logits<D, true>(se, ktile, kw, lane, ea, ec, 1.f, sturns, qb_ex, ka, kc);
+                    block_logits<D, true, RC>(sc, ktile, kw, lane, ra, rc, sturns, sdelta, qb_rm, ka, kc);
+                    block_logits<D, true, false>(se, ktile, kw, lane, ea, ec, sturns, sdelta, qb_ex, ka, kc);
                     if (ja >= j_exact) { sc[0] = se[0]; sc[1] = se[1]; }
                     if (jc >= j_exact) { sc[2] = se[2]; sc[3] = se[3]; }
                 }
@@ -879,9 +916,24 @@ cudaError_t plan_splits(const DecodeProblem& p, int units, Kern kern, int nthrea
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads, smem);
     if (occ < 1) occ = 1;
-    int ns = (nsm * occ) / units;
-    ns = max(1, min(ns, max_splits(p.Lcap)));
-    ns = min(ns, max(1, (p.L + 63) / 64));
+    // Split count with the least modelled time: ceil(CTAs / slots) waves, each
+    // as long as one CTA's keys plus a fixed cost per CTA (set-up, pipeline
+    // fill, partial write) worth kCtaFixedKeys keys.  A wave that leaves slots
+    // empty leaves whole SMs at half occupancy for its full length, so e.g. 64
+    // units on 296 slots take 9 splits (576 CTAs, two nearly full waves), not
+    // 4 (256 CTAs, 40 SMs with one CTA).  Ties go to fewer splits.
+    const long long slots = (long long)nsm * occ;
+    const int nsmax = max(1, min(max_splits(p.Lcap), (p.L + 63) / 64));
+    int ns = 1;
+    double best = 0.0;
+    for (int n = 1; n <= nsmax; ++n) {
+        const long long waves = ((long long)units * n + slots - 1) / slots;
+        const double t = (double)waves * ((double)p.L / n + kCtaFixedKeys);
+        if (n == 1 || t < best * 0.999) {
+            best = t;
+            ns = n;
+        }
+    }
     int chunk = (p.L + ns - 1) / ns;
     chunk = (chunk + gran - 1) / gran * gran;
     *ns_out = (p.L + chunk - 1) / chunk;
@@ -899,7 +951,10 @@ cudaError_t plan_scalar(const DecodeProblem& p, DecodeLaunch& dl)
 template <int D, int HPB>
 cudaError_t plan_tc(const DecodeProblem& p, DecodeLaunch& dl)
 {
-    return plan_splits(p, p.B * p.Hkv * dl.hgroups, decode_tc_kernel<D, HPB>, TC_NT,
+    if (p.rope_cache)
+        return plan_splits(p, p.B * p.Hkv * dl.hgroups, decode_tc_kernel<D, HPB, true>, TC_NT,
+                           DecTcCfg<D, HPB>::TOTAL, TC_KROWS, &dl.n_splits, &dl.chunk);
+    return plan_splits(p, p.B * p.Hkv * dl.hgroups, decode_tc_kernel<D, HPB, false>, TC_NT,
                        DecTcCfg<D, HPB>::TOTAL, TC_KROWS, &dl.n_splits, &dl.chunk);
 }
 
@@ -957,7 +1012,10 @@ cudaError_t launch_tc(const DecodeProblem& p, DecodeLaunch dl, cudaStream_t st)
     e = cudaMemsetAsync(dl.tickets, 0, sizeof(unsigned int) * (size_t)units, st);
     if (e != cudaSuccess) return e;
     dim3 grid(dl.n_splits, p.Hkv * dl.hgroups, p.B);
-    decode_tc_kernel<D, HPB><<<grid, TC_NT, DecTcCfg<D, HPB>::TOTAL, st>>>(tk, tv, p, dl);
+    if (p.rope_cache)
+        decode_tc_kernel<D, HPB, true><<<grid, TC_NT, DecTcCfg<D, HPB>::TOTAL, st>>>(tk, tv, p, dl);
+    else
+        decode_tc_kernel<D, HPB, false><<<grid, TC_NT, DecTcCfg<D, HPB>::TOTAL, st>>>(tk, tv, p, dl);
     return cudaGetLastError();
 }
 
