@@ -84,7 +84,15 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
  *   w0 >= 0 local window (w0 = 0: every pair remote; w0 >= L: every pair local);
  *   w_pretrained >= 1; rope_theta > 1; scale > 0 and finite.
  *   d must be 64 or 128 (else JETLONG_ERR_UNSUPPORTED); Hq % Hkv == 0.
- * Sizes: B*Hq*L*d < 2^31 per tensor is NOT required; L < 2^31. */
+ * Sizes: B*Hq*L*d < 2^31 per tensor is NOT required; L < 2^31.
+ * bf16 device memory: the call rotates every key once, to its exact and to its
+ * aliased position, into fp16 copies (B*Hkv*L*d*2 bytes each; one copy when
+ * G = 1) that the attention kernel loads tile by tile.  They live in a
+ * stream-ordered pool the library keeps per device: allocated and freed on
+ * `stream` around the kernels, reused by later calls, and reserved until the
+ * process exits.  If the pool cannot grow the call returns JETLONG_ERR_CUDA
+ * before any launch of the attention kernel.  The chunked, variable-length,
+ * three-pass and streamed calls do the same per launch. */
 int jetlong_prefill(const void* q, const void* k, const void* v, void* out,
                     int B, int Hq, int Hkv, int L, int d,
                     int w0, int w_pretrained, double rope_theta, float scale,
@@ -117,9 +125,9 @@ int jetlong_prefill_chunk(const void* q, const void* kcache, const void* vcache,
  *   aligned; row i of sequence b receives log sum_j exp(scale * logit_ij)
  *   (natural log; the statistic an LSE merge of partial attentions needs).
  * Other arguments and errors as jetlong_prefill.  bf16: one prefill launch
- * (after a range scan) per 64 sequences, its grid over the query blocks of all
- * of them, heaviest first; padding rows of q and k may hold anything.  fp32:
- * one launch per sequence. */
+ * (after a range scan and a key rotation) per 64 sequences, its grid over the
+ * query blocks of all of them, heaviest first; padding rows of q and k may
+ * hold anything.  fp32: one launch per sequence. */
 int jetlong_prefill_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                            int B, int Hq, int Hkv, const int32_t* lens, int Lmax, int d,
                            int w0, int w_pretrained, double rope_theta, float scale,

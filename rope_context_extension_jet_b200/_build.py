@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libjetlong.so")
 
-SOURCES = ["jetlong_api.cu", "position_map.cu", "range_scan.cu", "prefill_simt.cu", "prefill_tc.cu",
+SOURCES = ["jetlong_api.cu", "position_map.cu", "range_scan.cu", "rope_keys.cu", "prefill_simt.cu", "prefill_tc.cu",
            "prefill_pair.cu", "ie_merge.cu", "decode.cu", "debug_kernels.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",

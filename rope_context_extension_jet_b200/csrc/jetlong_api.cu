@@ -101,6 +101,34 @@ uint32_t* next_range_slot(cudaError_t* err)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Stream-ordered memory pool of this device for the pre-rotated keys of bf16
+// prefill calls.  It keeps what it has reserved (release threshold: all), so
+// after the first call of a given size the allocation needs no driver call;
+// the memory stays reserved by the pool until the process exits.
+cudaMemPool_t key_pool(cudaError_t* err)
+{
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        *err = cudaMemPoolCreate(&pool, &props);
+        if (*err != cudaSuccess) return nullptr;
+        uint64_t keep = ~0ull;
+        *err = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (*err != cudaSuccess) return nullptr;
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 int check_common(int B, int Hq, int Hkv, int d, int w0, int w_pretrained, double rope_theta,
                  float scale, jetlong_dtype dtype)
 {
@@ -232,11 +260,32 @@ static int prefill_entry(const void* q, const void* k, const void* v, void* out,
         p.range = slot;
     }
     take_injection(&p.inject, &p.wait_cycles);
-    // bf16: tensor-core kernel; fp32: CUDA-core fp32 kernel (TF32 would miss fp32 accuracy)
-    e = dtype == JETLONG_BF16 ? jl::launch_prefill_tc(p, (cudaStream_t)stream, &n)
-                              : jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
+    if (dtype != JETLONG_BF16) {
+        // fp32: CUDA-core fp32 kernel (TF32 would miss fp32 accuracy)
+        e = jl::launch_prefill_simt(p, dtype, (cudaStream_t)stream, &n);
+        g_launches += n;
+        if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    // bf16: the keys rotated once to their exact and aliased positions (fp16,
+    // in stream-ordered memory of the call), then the tensor-core kernel
+    cudaMemPool_t pool = key_pool(&e);
+    if (!pool) return fail(JETLONG_ERR_CUDA, "key pool: %s", cudaGetErrorString(e));
+    const size_t kbytes = (jl::rope_keys_bytes(p) + 255) & ~(size_t)255;
+    const bool remote = jl::rope_keys_need_remote(p);
+    void* kbuf = nullptr;
+    e = cudaMallocFromPoolAsync(&kbuf, remote ? 2 * kbytes : kbytes, pool, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "rotated-key buffer (%zu bytes): %s",
+                                      remote ? 2 * kbytes : kbytes, cudaGetErrorString(e));
+    p.krot_l = kbuf;
+    p.krot_r = remote ? static_cast<char*>(kbuf) + kbytes : kbuf;
+    e = jl::launch_rope_keys(p, kbuf, remote ? static_cast<char*>(kbuf) + kbytes : nullptr, (cudaStream_t)stream, &n);
+    if (e == cudaSuccess) e = jl::launch_prefill_tc(p, (cudaStream_t)stream, &n);
     g_launches += n;
+    // freed in stream order: the memory is reused only after the kernels above
+    const cudaError_t ef = cudaFreeAsync(kbuf, (cudaStream_t)stream);
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+    if (ef != cudaSuccess) return fail(JETLONG_ERR_CUDA, "rotated-key buffer release: %s", cudaGetErrorString(ef));
     return ok();
 }
 

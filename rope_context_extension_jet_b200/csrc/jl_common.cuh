@@ -118,6 +118,11 @@ struct PrefillProblem {
     int vl_len[64], vl_G[64];
     // bf16: write out as fp32 rows (the three-pass form's intermediate passes)
     int out_f32;
+    // bf16: the call's keys rotated once by launch_rope_keys, fp16 planes of L
+    // rows: to their exact positions (krot_l) and to floor(j / G) (krot_r,
+    // equal to krot_l when G = 1 throughout)
+    const void* krot_l;
+    const void* krot_r;
 };
 
 struct DecodeProblem {
@@ -182,5 +187,13 @@ struct ScanRows {
 cudaError_t launch_range_scan(const void* q, int C, int Cst, int q_planes, const void* k, int L, int Lcap,
                               int k_planes, int d, uint32_t* range, cudaStream_t s, int* nlaunch,
                               const ScanRows* rows = nullptr);
+
+// Keys of a bf16 prefill call rotated once to their exact and aliased
+// positions (rope_keys.cu): bytes of one fp16 copy, whether the aliased copy
+// differs from the exact one (some G > 1), and the launch that writes kl (and
+// kr unless null) after the call's range scan on the same stream.
+size_t rope_keys_bytes(const PrefillProblem& p);
+bool rope_keys_need_remote(const PrefillProblem& p);
+cudaError_t launch_rope_keys(const PrefillProblem& p, void* kl, void* kr, cudaStream_t s, int* nlaunch);
 
 }  // namespace jl

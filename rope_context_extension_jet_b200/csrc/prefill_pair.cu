@@ -5,31 +5,34 @@
 // "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
 // (gist.science/it/paper/2607.07740), Metodologia 1-2: local pairs
 // (i - j < w0) are rotated at (i, j), remote pairs at (floor(i/G), floor(j/G)),
-// rotations applied on the fly to the raw inputs, one softmax for both.
+// one softmax for both.  The keys come rotated both ways, once per call
+// (rope_keys.cu: fp16 copies at j and at floor(j/G)); Q is rotated here.
 //
 // Work unit of a pair: one block of 128 query rows of the four query heads
 // that share a kv head.  CTA r (r = 0, 1) holds heads 2r and 2r + 1 of the four:
 // their Q tiles, S and O in its own TMEM (lanes = query rows).  A K tile (128
-// keys) is split by keys: CTA r loads and rotates keys [64r, 64r + 64); a V tile
-// is split by columns: CTA r loads V[:, 64r, 64r + 64).  One MMA
+// keys) is split by keys: CTA r loads keys [64r, 64r + 64) of the copy the
+// tile's phase uses; a V tile is split by columns: CTA r loads
+// V[:, 64r, 64r + 64).  One MMA
 //   S_h = Q_h K^T : A = Q_h of both CTAs (M = 256), B = both K halves (N = 128)
 //   O_h += P_h V  : A = P_h in both TMEMs, B = both V halves (N = d)
-// so each SM stages and rotates half of every K/V tile, and reads half of the
-// B operand from its shared memory, while the MMA rate per SM is unchanged.
+// so each SM stages half of every K/V tile, and reads half of the B operand
+// from its shared memory, while the MMA rate per SM is unchanged.
 // The phases, masks and softmax are those of the one-CTA kernel
 // (prefill_tc.cu): phase R (remote and band tiles, aliased positions), then
 // phase E (band and local tiles, exact positions), Q re-rotated in between.
 //
 // Roles (512 threads per CTA; registers rebalanced with setmaxnreg):
-//   warp 0      TMA producer (both CTAs): own Q tiles, own K and V halves
+//   warp 0      TMA producer (both CTAs): own Q tiles, own K (rotated copy of
+//               the tile's phase) and V halves
 //   warp 1      MMA issuer (CTA 0 only; the whole warp runs the loop, one
 //               elected lane issues each instruction), cta_group::2
 //   warp 2      TMEM allocation / release (cta_group::2, both CTAs)
 //   warp 3      CTA 1: tells CTA 0 when its V half landed
-//   warps 4-7   rotation of own Q tiles and own K halves
+//   warps 4-7   rotation of own Q tiles; pass each landed K half on to CTA 0
 //   warps 8-15  softmax, heads 2r (8-11) and 2r + 1 (12-15)
 // Synchronisation: CTA 0's MMA thread waits on barriers in CTA 0 that both CTAs
-// arrive on (Q and K rotated, P written, V halves landed); its commits arrive
+// arrive on (Q rotated, K halves landed, P written, V halves landed); its commits arrive
 // on the barriers at the same offset in both CTAs (S ready, P.V done, buffers
 // free).  Every wait is bounded; on expiry a CTA records an error code, stops,
 // and both CTAs meet at the closing cluster barrier before TMEM is released.
@@ -73,8 +76,9 @@ struct PairSmem {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const TcParams p)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKl,
+                        const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmV,
+                        const TcParams p)
 {
     using S = PairSmem;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -151,7 +155,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmKl);
+            tma_prefetch_desc(&tmKr);
             tma_prefetch_desc(&tmV);
             const int zkv = b * p.Hkv + kvh;
             mbar_arrive_expect_tx(&bars[P_QFULL], 2 * S::QTILE);
@@ -166,9 +171,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 const int s = e % NS, u = e / NS;
                 if (e >= NS && !wait_or_abort<true>(&bars[P_KEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x401)) break;
                 mbar_arrive_expect_tx(&bars[P_KFULL + s], S::KTILE);
+                // keys rotated to floor(j / G) in phase R (and in a windowed
+                // pass at the aliased positions), to j in phase E
+                const CUtensorMap* km = (e < nR || p.window_rot == 1) ? &tmKr : &tmKl;
 #pragma unroll
                 for (int a = 0; a < 2; ++a)
-                    tma_load_3d(smem + S::K0 + s * S::KTILE + a * S::KATOM, &tmK, a * 64, kb * BN + (int)rank * KROWS,
+                    tma_load_3d(smem + S::K0 + s * S::KTILE + a * S::KATOM, km, a * 64, kb * BN + (int)rank * KROWS,
                                 zkv, &bars[P_KFULL + s]);
                 k_issued = e + 1;
                 if (e >= NS && !wait_or_abort<true>(&bars[P_VEMPTY + s], (u - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x402)) break;
@@ -265,7 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
         // operand scales of this call (powers of two, see range_exp)
-        const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
+        const float lq = pow2i(range_exp(ld_range(p.range)));
         const uint32_t i0 = (uint32_t)(p.P + qb * BM);
         bool ok = warp_wait(&bars[P_QFULL], 0, abort_flag, p.dev_error, p.wait_cycles, 0x431);
         if (ok) {
@@ -281,7 +289,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (lane == 0) mbar_arrive_cluster(lead(P_QREADY0));
         }
         for (int e = 0; e < NE && ok; ++e) {
-            const int kb = tp.kb(e);
             const int s = e % NS, u = e / NS;
             if (e == nR && nR > 0) {
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
@@ -293,14 +300,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(lead(P_QREADY1));
             }
+            // the K half-tile arrives rotated (rope_keys.cu): pass its arrival on
+            // to the leader's MMA warp
             if (!warp_wait(&bars[P_KFULL + s], u & 1, abort_flag, p.dev_error, p.wait_cycles, 0x433)) { ok = false; break; }
-            const uint32_t j0 = (uint32_t)(kb * BN) + rank * KROWS;
-            unsigned char* kt = smem + S::K0 + s * S::KTILE;
-            if (e < nR || p.window_rot == 1)
-                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return div_g(j0 + r, sv); }, stc, sts, lk);
-            else
-                rotate_tile<D, KROWS, true, true>(kt, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
-            fence_proxy_async_smem();
             __syncwarp();
             // (test hook: the first key tile is never released, so the MMA warp's
             // bounded wait on it expires)
@@ -329,10 +331,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
 cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
 {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tkl, tkr, tv;
     cudaError_t e;
     if ((e = make_map(&tq, pp.q, D, pp.C, pp.Cst, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, KROWS)) != cudaSuccess) return e;
+    if ((e = make_map(&tkl, pp.krot_l, D, pp.L, pp.L, pp.B * pp.Hkv, KROWS, true)) != cudaSuccess) return e;
+    if ((e = make_map(&tkr, pp.krot_r, D, pp.L, pp.L, pp.B * pp.Hkv, KROWS, true)) != cudaSuccess) return e;
     if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);
     constexpr int smem = PairSmem::TOTAL;
@@ -341,7 +344,7 @@ cudaError_t launch_prefill_pair(const PrefillProblem& pp, cudaStream_t st)
         return e;
     // variable-length: x over (query-block level, sequence), one z
     dim3 grid(p.vl_n ? 2 * p.vl_nqb_max * p.vl_n : 2 * p.nqb, pp.Hq / 4, p.vl_n ? 1 : pp.B);
-    prefill_pair_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
+    prefill_pair_kernel<<<grid, NTHREADS, smem, st>>>(tq, tkl, tkr, tv, p);
     return cudaGetLastError();
 }
 

@@ -5,14 +5,16 @@
 // (gist.science/it/paper/2607.07740):
 //   Metodologia 1 -- a pair (i, j) with i - j < w0 uses classic RoPE at i and
 //   j; every other pair uses RoPE at f(i), f(j), f(x) = floor(x / G).
-//   Metodologia 2 -- rotations are applied on the fly to unrotated inputs
-//   (they compose additively) and all routed pairs feed one exact softmax.
+//   Metodologia 2 -- rotations compose additively, and all routed pairs feed
+//   one exact softmax.
 //   The pages merge three FlashAttention passes by inclusion-exclusion; here
 //   one pass computes the routed logits directly.
 //
 // Work unit: 128 query rows of NH = 2 query heads that share a kv head
-// (grouped-query attention), so every raw K tile is loaded and rotated once
-// for both heads.  Each CTA makes two passes over its key tiles (128 keys):
+// (grouped-query attention), so every K tile is loaded once for both heads.
+// The keys come rotated once per call (rope_keys.cu: fp16 copies at j and at
+// floor(j/G)); each tile is loaded from the copy of its phase.  Each CTA makes
+// two passes over its key tiles (128 keys):
 //   phase R -- tiles holding remote pairs (remote-only and band tiles), with Q
 //              and K rotated to the aliased positions floor(x / G);
 //   phase E -- tiles holding local pairs (band and local-only tiles), with Q
@@ -23,13 +25,14 @@
 // (rotations compose additively).
 //
 // Warp roles (512 threads, 4 warpgroups; registers rebalanced with setmaxnreg):
-//   warp 0        TMA producer (raw Q once; raw K and V per tile)
+//   warp 0        TMA producer (raw Q once; rotated K and V per tile)
 //   warp 1        MMA issuer (the whole warp; one elected lane issues each
 //                 group of MMAs): S_h = Q_h K^T (fp16 operands) into TMEM;
 //                 O_h += P_h V with P_h read from TMEM (bf16)
 //   warp 2        TMEM allocation / release
-//   warps 4-7     rotation: RoPE of Q and of every K tile in shared memory,
-//                 angles advanced row by row with a per-frequency rotation step
+//   warps 4-7     rotation: RoPE of Q in shared memory, angles advanced row by
+//                 row with a per-frequency rotation step; then the arrival of
+//                 each K tile is passed on to the MMA warp
 //   warps 8-11    softmax for head 0, warps 12-15 for head 1: one thread per
 //                 query row (= TMEM lane); causal / length / band masks, online
 //                 softmax in base 2 with lazy O rescaling, P (bf16) back into
@@ -79,8 +82,9 @@ struct TcSmem {
 
 template <int D, int NH>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const TcParams p)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKl,
+                      const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmV,
+                      const TcParams p)
 {
     using S = TcSmem<D, NH>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -146,7 +150,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------------- TMA producer
             tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmKl);
+            tma_prefetch_desc(&tmKr);
             tma_prefetch_desc(&tmV);
             const int zkv = b * p.Hkv + kvh;
             mbar_arrive_expect_tx(&bars[B_QFULL], NH * S::TILE);
@@ -161,9 +166,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int sk = e % NSK, uk = e / NSK;
                 if (e >= NSK && !wait_or_abort(&bars[B_KEMPTY + sk], (uk - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x301)) break;
                 mbar_arrive_expect_tx(&bars[B_KFULL + sk], S::TILE);
+                // keys rotated to floor(j / G) in phase R (and in a windowed
+                // pass at the aliased positions), to j in phase E
+                const CUtensorMap* km = (e < nR || p.window_rot == 1) ? &tmKr : &tmKl;
 #pragma unroll
                 for (int a = 0; a < S::ATOMS; ++a)
-                    tma_load_3d(smem + S::K0 + sk * S::TILE + a * ATOM, &tmK, a * 64, kb * BN, zkv, &bars[B_KFULL + sk]);
+                    tma_load_3d(smem + S::K0 + sk * S::TILE + a * ATOM, km, a * 64, kb * BN, zkv, &bars[B_KFULL + sk]);
                 k_issued = e + 1;
                 const int sv = e % NSV, uv = e / NSV;
                 if (e >= NSV && !wait_or_abort(&bars[B_VEMPTY + sv], (uv - 1) & 1, abort_flag, p.dev_error, p.wait_cycles, 0x302)) break;
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float2 stc[4], sts[4];  // per-frequency one-position step R(theta_m)
         rope_steps<D>(t, p, stc, sts);
         // operand scales of this call (powers of two, see range_exp)
-        const float lq = pow2i(range_exp(ld_range(p.range))), lk = pow2i(range_exp(ld_range(p.range + 1)));
+        const float lq = pow2i(range_exp(ld_range(p.range)));
         const uint32_t i0 = (uint32_t)(p.P + qb * BM);
         bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.dev_error, p.wait_cycles, 0x321);
         if (ok) {
@@ -275,7 +283,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0) mbar_arrive(&bars[B_QREADY0]);
         }
         for (int e = 0; e < NE && ok; ++e) {
-            const int kb = tp.kb(e);
             const int sk = e % NSK, uk = e / NSK;
             if (e == nR && nR > 0) {
                 // phase switch: Q from floor(i/G) to i, by the extra rotation i - floor(i/G)
@@ -287,14 +294,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_QREADY1]);
             }
+            // the K tile arrives rotated (rope_keys.cu): pass its arrival on
             if (!warp_wait(&bars[B_KFULL + sk], uk & 1, abort_flag, p.dev_error, p.wait_cycles, 0x323)) { ok = false; break; }
-            const uint32_t j0 = (uint32_t)(kb * BN);
-            if (e < nR || p.window_rot == 1)
-                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return div_g(j0 + r, sv); }, stc,
-                                         sts, lk);
-            else
-                rotate_tile<D, BM, true, false>(smem + S::K0 + sk * S::TILE, t, p, [&](int r) { return j0 + r; }, stc, sts, lk);
-            fence_proxy_async_smem();
             __syncwarp();
             // (test hook: the first key tile is never released, so the MMA
             // thread's bounded wait on it expires)
@@ -325,10 +326,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 template <int D, int NH>
 cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
 {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tkl, tkr, tv;
     cudaError_t e;
     if ((e = make_map(&tq, pp.q, D, pp.C, pp.Cst, pp.B * pp.Hq, BM)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, pp.k, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
+    if ((e = make_map(&tkl, pp.krot_l, D, pp.L, pp.L, pp.B * pp.Hkv, BN, true)) != cudaSuccess) return e;
+    if ((e = make_map(&tkr, pp.krot_r, D, pp.L, pp.L, pp.B * pp.Hkv, BN, true)) != cudaSuccess) return e;
     if ((e = make_map(&tv, pp.v, D, pp.L, pp.Lcap, pp.B * pp.Hkv, BN)) != cudaSuccess) return e;
     const TcParams p = make_params(pp);
     auto kern = prefill_tc_kernel<D, NH>;
@@ -337,7 +339,7 @@ cudaError_t launch_d(const PrefillProblem& pp, cudaStream_t st)
         return e;
     // variable-length: x over (query-block level, sequence), one z
     dim3 grid(p.vl_n ? p.vl_nqb_max * p.vl_n : p.nqb, pp.Hq / NH, p.vl_n ? 1 : pp.B);
-    kern<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, tkl, tkr, tv, p);
     return cudaGetLastError();
 }
 
@@ -374,7 +376,7 @@ void make_div_magic(uint32_t G, uint32_t* m, uint32_t* s1, uint32_t* s2)
 }  // namespace
 
 cudaError_t make_map(CUtensorMap* m, const void* base, int d, int rows, int plane_rows, int nplanes,
-                     int box_rows)
+                     int box_rows, bool f16)
 {
     cudaError_t err;
     EncodeTiledFn fn = encode_fn(&err);
@@ -383,7 +385,8 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int d, int rows, int plan
     const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)plane_rows * d * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+    CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void*>(base), dims, strides, box,
                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;

@@ -479,10 +479,11 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const SeqView& s
 
 // ------------------------------------------------------------------ host side
 
-// [planes][plane_rows][d] bf16 read as rows [0, rows) of every plane (rows >=
-// rows load as zeros), box 64 columns x box_rows rows x 1 plane, 128-byte swizzle.
+// [planes][plane_rows][d] bf16 (fp16 when f16) read as rows [0, rows) of every
+// plane (rows >= rows load as zeros), box 64 columns x box_rows rows x 1 plane,
+// 128-byte swizzle.
 cudaError_t make_map(CUtensorMap* m, const void* base, int d, int rows, int plane_rows, int nplanes,
-                     int box_rows);
+                     int box_rows, bool f16 = false);
 
 // Parameters shared by both kernels (G magic numbers, RoPE turns, output).
 TcParams make_params(const PrefillProblem& pp);

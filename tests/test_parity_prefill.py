@@ -304,14 +304,14 @@ def test_varlen_lengths_cross_group_sizes():
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 2), (2, 2)])
 def test_varlen_one_launch_for_64_sequences(Hq, Hkv):
-    # bf16: one range scan + one prefill launch per 64 sequences (70 here: two
-    # of each), every sequence with its own length and G; NaN in the padding
-    # rows of q and k must not reach any output
+    # bf16: one range scan, one key rotation and one prefill launch per 64
+    # sequences (70 here: two of each), every sequence with its own length and
+    # G; NaN in the padding rows of q and k must not reach any output
     rng = np.random.default_rng(74)
     lens = [int(x) for x in rng.integers(1, 300, size=70)]
     lens[3], lens[40] = 300, 129
     varlen_case("varlen-70", lens, Hq=Hq, Hkv=Hkv, w_pre=64, w0=40, index=74, nan_qk_padding=True,
-                launches=4)
+                launches=6)
 
 
 # ---------------------------------------------------------------- inclusion-exclusion form
