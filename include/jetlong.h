@@ -285,11 +285,20 @@ int jetlong_debug_inject_timeout(int site, long long wait_cycles);
  * exact-phase tiles [kE0, nkb) -- and d_cls[qb max_kb + kb] (kb < min(nkb,
  * max_kb)) the class of tile (qb, kb): 0 every causal pair remote, 1 every pair
  * local, 2 both.  Device arrays of 3 ceil(C / 128) int32 and ceil(C / 128)
- * max_kb int8.  Both return JETLONG_OK, JETLONG_ERR_INVALID_ARG or
- * JETLONG_ERR_CUDA; asynchronous on stream. */
+ * max_kb int8.
+ *
+ * jetlong_debug_ex2: d_out[i] = 2^d_y[i] as the one-CTA prefill's softmax
+ * forms part of its exponentials on the FMA pipe (round to an integer n,
+ * cubic in the remainder, exponent bits for 2^n; inputs below -127 give 0,
+ * NaN stays NaN).  Meant for y <= 2^7, the softmax's range.  d_y, d_out:
+ * device float arrays of n elements, n even.
+ *
+ * All return JETLONG_OK, JETLONG_ERR_INVALID_ARG or JETLONG_ERR_CUDA;
+ * asynchronous on stream. */
 int jetlong_debug_rope_phase(const uint32_t* d_pos, int64_t n, int d, double rope_theta, int accurate,
                              float* d_out, void* stream);
 int jetlong_debug_tile_plan(int P, int C, int w0, int max_kb, int32_t* d_plan, int8_t* d_cls, void* stream);
+int jetlong_debug_ex2(const float* d_y, int64_t n, float* d_out, void* stream);
 
 /* Message for the last failing call on this host thread ("" if none). */
 const char* jetlong_last_error(void);

@@ -24,7 +24,7 @@ __all__ = [
     "prefill_chunk", "prefill_varlen", "prefill_ie", "prefill_streamed", "decode_workspace_size",
     "decode", "decode_rope_cache", "decode_noalloc", "device_status", "last_error", "launch_count",
     "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout", "debug_inject_timeout",
-    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY", "debug_rope_phase", "debug_tile_plan",
+    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY", "debug_rope_phase", "debug_tile_plan", "debug_ex2",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +95,8 @@ def load_library(path: str | None = None):
         lib.jetlong_debug_rope_phase.argtypes = [vp, i64, i32, dbl, i32, vp, vp]
         lib.jetlong_debug_tile_plan.restype = i32
         lib.jetlong_debug_tile_plan.argtypes = [i32, i32, i32, i32, vp, vp, vp]
+        lib.jetlong_debug_ex2.restype = i32
+        lib.jetlong_debug_ex2.argtypes = [vp, i64, vp, vp]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -431,6 +433,20 @@ def debug_tile_plan(P: int, C: int, w0: int, max_kb: int, stream=None):
     _check(lib.jetlong_debug_tile_plan(int(P), int(C), int(w0), int(max_kb), _dev(plan, "plan"), _dev(cls, "cls"),
                                        _stream(stream)), lib)
     return plan, cls
+
+
+def debug_ex2(y, stream=None):
+    """2^y as the one-CTA prefill's softmax forms part of its exponentials on the
+    FMA pipe (test hook jetlong_debug_ex2).  y: float32 CUDA tensor with an even
+    number of elements; returns a tensor of the same shape."""
+    import torch
+    if y.dtype != torch.float32 or y.numel() % 2:
+        raise TypeError("y must be float32 with an even number of elements")
+    y = y.contiguous()
+    out = torch.empty_like(y)
+    lib = load_library()
+    _check(lib.jetlong_debug_ex2(_dev(y, "y"), y.numel(), _dev(out, "out"), _stream(stream)), lib)
+    return out
 
 
 def device_status(stream=None):

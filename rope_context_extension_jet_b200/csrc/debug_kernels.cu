@@ -1,7 +1,8 @@
 // debug_kernels.cu -- test hooks that run the device helpers of the attention
 // kernels on their own, so tests can check them against independent host
-// computations: the RoPE phase (fixed-point turns, then sin / cos) and the
-// prefill's tile classification and per-query-block tile plan.
+// computations: the RoPE phase (fixed-point turns, then sin / cos), the
+// prefill's tile classification and per-query-block tile plan, and the
+// softmax's exponential on the FMA pipe.
 #include "prefill_tc_common.cuh"
 
 namespace jl {
@@ -41,7 +42,27 @@ __global__ void tile_plan_kernel(int P, int C, int L, int w0, int max_kb, int32_
         cls[(long long)qb * max_kb + kb] = (int8_t)tc::tile_class(i_lo, kb, L, w0);
 }
 
+// out[i] = ex2_poly2(y[i]) (pairs of consecutive elements; n even)
+__global__ void ex2_poly_kernel(const float* y, long long n, float* out)
+{
+    const long long e = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (e + 1 >= n) return;
+    const float2 r = tc::ex2_poly2(make_float2(y[e], y[e + 1]));
+    out[e] = r.x;
+    out[e + 1] = r.y;
+}
+
 }  // namespace
+
+cudaError_t launch_ex2_poly(const float* y, long long n, float* out, cudaStream_t s, int* nlaunch)
+{
+    const long long pairs = n / 2;
+    if (pairs <= 0) return cudaSuccess;
+    ex2_poly_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(y, n, out);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) *nlaunch += 1;
+    return e;
+}
 
 cudaError_t launch_rope_phase(const uint32_t* pos, long long n, int d, const RopeTurns& turns, int accurate,
                               float* out, cudaStream_t s, int* nlaunch)

@@ -669,6 +669,17 @@ int jetlong_debug_tile_plan(int P, int C, int w0, int max_kb, int32_t* d_plan, i
     return ok();
 }
 
+int jetlong_debug_ex2(const float* d_y, int64_t n, float* d_out, void* stream)
+{
+    if (!d_y || !d_out) return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (n < 0 || (n & 1)) return fail(JETLONG_ERR_INVALID_ARG, "need an even n >= 0 (got %lld)", (long long)n);
+    int nl = 0;
+    cudaError_t e = jl::launch_ex2_poly(d_y, n, d_out, (cudaStream_t)stream, &nl);
+    g_launches += nl;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "ex2 launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 int jetlong_device_status(void* stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

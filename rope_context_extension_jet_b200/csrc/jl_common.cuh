@@ -176,6 +176,7 @@ cudaError_t launch_wait_selftest(int* dev_error, long long limit_cycles, cudaStr
 // Test hooks (debug_kernels.cu): the phase helpers and the tile plan on their own.
 cudaError_t launch_rope_phase(const uint32_t* pos, long long n, int d, const RopeTurns& turns, int accurate,
                               float* out, cudaStream_t s, int* nlaunch);
+cudaError_t launch_ex2_poly(const float* y, long long n, float* out, cudaStream_t s, int* nlaunch);
 cudaError_t launch_tile_plan(int P, int C, int L, int w0, int max_kb, int32_t* plan, int8_t* cls, cudaStream_t s,
                              int* nlaunch);
 // rows (optional): per-sequence row counts of a variable-length batch, plane pl

@@ -25,6 +25,11 @@ constexpr int BM = 128, BN = 128;
 constexpr int kVarlenMax = 64;  // sequences of one variable-length launch
 constexpr int ATOM = 128 * 128;  // bytes of one 128-row x 64-column 16-bit swizzle atom
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+// softmax exponentials of the one-CTA kernel: one pair in every
+// kPolyExpPeriod groups of four columns goes to ex2_poly2 (FMA pipe), the rest
+// to the MUFU.  (The CTA-pair kernel measured no gain from it: all its
+// exponentials use the MUFU.)
+constexpr int kPolyExpPeriod = 2;
 
 enum { CLS_REM = 0, CLS_LOC = 1, CLS_BAND = 2 };
 
@@ -117,6 +122,34 @@ __device__ __forceinline__ uint32_t ld_range(const uint32_t* p)
     uint32_t v;
     asm volatile("ld.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
+}
+
+// 2^y for a pair y (y <= 2^7) on the FMA and integer pipes, sparing the MUFU
+// that evaluates the other exponentials of the softmax.  y = n + f with
+// n = round(y) (adding 1.5 * 2^23 rounds to an integer held in the low bits)
+// and f in [-1/2, 1/2]; 2^f by a cubic fitted to 2^f over that interval for the
+// least largest relative error (7.5e-5, against 2^-9 for the bf16 rounding of
+// P); 2^n from the exponent field n + 127.  y is first raised to -127 by a
+// max that keeps NaN: there the exponent field is 0, so -inf gives exactly 0,
+// and a NaN stays NaN.
+__device__ __forceinline__ float2 ex2_poly2(float2 y)
+{
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    constexpr float C0 = 0.99992806f, C1 = 0.69326097f, C2 = 0.24261114f, C3 = 0.055171669f;
+    float a, b;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(a) : "f"(y.x), "f"(-127.f));
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(b) : "f"(y.y), "f"(-127.f));
+    const float2 yc = make_float2(a, b);
+    const float2 t = add2(yc, make_float2(kRound, kRound));
+    const float2 n = add2(t, make_float2(-kRound, -kRound));
+    const float2 f = fma2(n, make_float2(-1.f, -1.f), yc);  // exact: y - n
+    float2 p = fma2(make_float2(C3, C3), f, make_float2(C2, C2));
+    p = fma2(p, f, make_float2(C1, C1));
+    p = fma2(p, f, make_float2(C0, C0));
+    // low bits of t hold n (two's complement); (n + 127) << 23 is 2^n
+    const float2 s = make_float2(__uint_as_float((__float_as_uint(t.x) + 127u) << 23),
+                                 __uint_as_float((__float_as_uint(t.y) + 127u) << 23));
+    return mul2(p, s);
 }
 
 __device__ __forceinline__ uint32_t div_g(uint32_t n, const SeqView& v)
@@ -404,7 +437,10 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, const SeqView& s
                 const float2 y0 = fma2(make_float2(x[u], x[u + 1]), sl, nm);
                 const float2 y1 = fma2(make_float2(x[u + 2], x[u + 3]), sl, nm);
                 const float2 p0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-                const float2 p1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+                // one-CTA kernel: one pair in every kPolyExpPeriod steps of 4 on the FMA pipe
+                const float2 p1 = !CLUSTER && (v / 4) % kPolyExpPeriod == kPolyExpPeriod - 1
+                                      ? ex2_poly2(y1)
+                                      : make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
                 acc0 = add2(acc0, p0);
                 acc1 = add2(acc1, p1);
                 pk[v >> 1] = pack_bf16x2(p0.x, p0.y);

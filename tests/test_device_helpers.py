@@ -13,6 +13,11 @@ through a test hook and checked against an independent host computation.
   class against brute-force classification of its causal pairs (local iff
   i - j < w0, Metodologia 1), and the plan's two phases against the sets of key
   blocks holding remote and local pairs.
+* Softmax exponential on the FMA pipe (jetlong_debug_ex2): 2^y as a quarter of
+  the one-CTA prefill's exponentials are formed, against numpy's exp2 in fp64
+  over the softmax's range (relative error <= 1e-4, well below the 2^-9 of
+  the bf16 P it feeds), with -inf and values below -127 giving exactly 0 and
+  NaN staying NaN.
 """
 import numpy as np
 import pytest
@@ -94,3 +99,26 @@ def test_tile_plan_against_brute_force(P, C, w0):
         local = {kb for kb, c in row.items() if c in (1, 2)}
         assert remote == set(range(nR)), (qb, nR, sorted(remote))
         assert local == set(range(kE0, nkb)), (qb, kE0, nkb, sorted(local))
+
+
+def test_softmax_exp2_on_fma_pipe():
+    import torch
+    rng = np.random.default_rng(91)
+    y = np.concatenate([np.linspace(-125.5, 8.0, 400001), rng.uniform(-30.0, 0.0, 100000),
+                        np.arange(-125, 9, dtype=np.float64), np.arange(-125, 8) + 0.5,
+                        np.array([0.0, -0.0, -1e-7, -0.5, 0.5, 7.999])]).astype(np.float32)
+    if y.size % 2:
+        y = np.append(y, np.float32(-1.0))
+    got = jl.debug_ex2(torch.from_numpy(y).cuda())
+    jl.device_status()
+    got = got.double().cpu().numpy()
+    ref = np.exp2(y.astype(np.float64))
+    rel = np.abs(got / ref - 1.0)
+    assert rel.max() <= 1e-4, f"relative error {rel.max():.3e} at y = {y[rel.argmax()]}"
+    # below the normal range of the result: tiny, and exactly 0 from -127 down
+    low = np.array([-126.0, -126.4, -126.6, -127.0, -128.0, -1000.0, -np.inf, np.nan], dtype=np.float32)
+    gl = jl.debug_ex2(torch.from_numpy(low).cuda()).double().cpu().numpy()
+    jl.device_status()
+    assert np.all(np.abs(gl[:3]) <= 2.0 ** -125)
+    assert np.all(gl[3:7] == 0.0), gl
+    assert np.isnan(gl[7])
