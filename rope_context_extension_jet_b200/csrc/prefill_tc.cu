@@ -76,7 +76,7 @@ struct TcSmem {
     static constexpr int K0 = NH * TILE;
     static constexpr int V0 = K0 + NSK * TILE;
     static constexpr int BAR = V0 + NSV * TILE;
-    static constexpr int END = BAR + NBARS * 8 + 16;
+    static constexpr int END = BAR + NBARS * 8 + 32;  // + TMEM slot, abort flag, tile plan
     static constexpr int TOTAL = END + 1024;  // slack to align the base to 1024
 };
 
