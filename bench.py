@@ -435,6 +435,36 @@ def _ncu_cmd(extra, bench_args, log):
             + [sys.executable, os.path.join(ROOT, "bench.py")] + bench_args)
 
 
+# Every capture profiles/ holds, in the order they run: (mode, L).
+NCU_ALL = (("launches", None), ("traffic", 131072), ("prefill", 32768), ("decode", 32768),
+           ("prefill-full", 32768), ("decode-full", 32768))
+
+
+def ncu_summary_name(mode, L):
+    """File name (without extension) under profiles/ of the capture `mode` at length L."""
+    if mode == "launches":
+        return "launches_bench"
+    kname = NCU_KERNELS["decode" if mode.startswith("decode") else "prefill"]
+    if mode == "traffic":
+        return f"{kname}_L{L}_dram"
+    if mode.endswith("-full"):
+        return f"{kname}_L{L}_full"
+    return f"{kname}_L{L}_counters"
+
+
+def run_ncu_all():
+    """Regenerate every summary under profiles/: each capture in its own process
+    (each runs its command plainly first, then under ncu); stops at the first
+    that fails."""
+    for mode, L in NCU_ALL:
+        cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--ncu", mode]
+        if L is not None:
+            cmd += ["--L", str(L)]
+        r = subprocess.run(cmd)
+        if r.returncode != 0:
+            raise SystemExit(f"capture {mode} exited {r.returncode}")
+
+
 def run_ncu(args):
     """Profiling harness: run the bench command once without ncu (it must exit 0),
     then the same command under ncu, and write the summary under profiles/."""
@@ -483,7 +513,7 @@ def run_ncu(args):
         lines += [f"| `{k}` | {n} | {t:.3f} | {sh:.1%} |" for k, n, t, sh in summ]
         rec = {"launches": [{"kernel": k, "launches": n, "total_ms": round(t, 4), "share": round(sh, 4)}
                             for k, n, t, sh in summ]}
-        name = "launches_bench"
+        name = ncu_summary_name("launches", None)
     else:
         m = {r["metric"]: r["value"] for r in rows}
         if args.ncu.endswith("-full"):
@@ -507,12 +537,7 @@ def run_ncu(args):
             rec["frac_of_hbm"] = rec["gbs_kv"] / peaks["hbm_gbs"] if rec["gbs_kv"] else None
             kname = NCU_KERNELS["decode"]
         rec["peaks"] = {k: v for k, v in peaks.items()}
-        if args.ncu == "traffic":
-            name = f"{kname}_L{args.L}_dram"
-        elif args.ncu.endswith("-full"):
-            name = f"{kname}_L{args.L}_full"
-        else:
-            name = f"{kname}_L{args.L}_counters"
+        name = ncu_summary_name(args.ncu, args.L)
         lines += [f"# `{kname}`: {rec['workload']}", "", "One launch after one warm-up launch (ncu, clock control none),",
                   "captured after the same command exited 0 without ncu:", "", "    " + shown, "",
                   "| metric | value |", "|---|---|"]
@@ -528,12 +553,16 @@ def run_ncu(args):
                           f"({peaks['hbm_gbs']} GB/s); DRAM counted {dram / 1e9:.3f} GB."]
     srcs = DECODE_SOURCES if args.ncu.startswith("decode") else PREFILL_SOURCES
     if args.ncu == "launches":
-        srcs = PREFILL_SOURCES + ("decode.cu", "range_scan.cu")
+        srcs = PREFILL_SOURCES + ("decode.cu", "range_scan.cu", "rope_keys.cu")
     lines += ["", f"Sources: sha256 of {', '.join(srcs)}: {prefill_source_hash(srcs)[:16]}; "
                   f"capture took {secs:.0f} s."]
     prof = os.path.join(ROOT, "profiles")
     with open(os.path.join(prof, name + ".md"), "w") as f:
         f.write("\n".join(lines) + "\n")
+    rec["command"] = shown
+    rec["sources"] = {"files": list(srcs), "sha256": prefill_source_hash(srcs)}
+    with open(os.path.join(prof, name + ".json"), "w") as f:
+        json.dump(rec, f, indent=1, sort_keys=True)
     if args.ncu == "traffic" and args.L == I.C4.L:
         tr_path = os.path.join(prof, "traffic.json")
         try:
@@ -559,11 +588,13 @@ def main():
     ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
                     help="run only one kernel on a reduced workload (for ncu captures)")
     ap.add_argument("--L", type=int, default=32768, help="sequence / cache length for --profile")
-    ap.add_argument("--ncu", choices=["launches", "prefill", "decode", "traffic", "prefill-full", "decode-full"],
+    ap.add_argument("--ncu", choices=["launches", "prefill", "decode", "traffic", "prefill-full", "decode-full",
+                                      "all"],
                     default=None,
                     help="profiling harness: the bench command (launches), one kernel of the --profile "
                          "workloads (prefill, decode) or one full-size prefill's DRAM bytes (traffic, "
-                         "--L 131072), under ncu; writes the summary under profiles/")
+                         "--L 131072), under ncu; writes the summary (.md) and its figures (.json) under "
+                         "profiles/; 'all' runs every capture profiles/ holds, one after the other")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -573,6 +604,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.ncu == "all":
+        run_ncu_all()
         return
     if args.ncu:
         run_ncu(args)

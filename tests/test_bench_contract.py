@@ -2,6 +2,7 @@
 kernel time into TFLOP/s (against brute force over the (query, key) pairs),
 and the JSON line of the CPU-oracle arm (`--impl reference`)."""
 import io
+import os
 import json
 import types
 from contextlib import redirect_stdout
@@ -131,3 +132,13 @@ def test_ncu_raw_csv_parsing():
     m = {r["metric"]: r["value"] for r in rows}
     assert m["gpu__time_duration.sum"] == 8708000.0 and m["dram__bytes_read.sum"] == 404577000.0
     assert rows[0]["kernel"].startswith("prefill_pair_kernel")
+
+
+def test_ncu_all_regenerates_every_committed_profile():
+    # one command (bench.py --ncu all) makes every summary profiles/ holds
+    made = {bench.ncu_summary_name(mode, L) for mode, L in bench.NCU_ALL}
+    prof = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles")
+    for f in os.listdir(prof):
+        stem, ext = os.path.splitext(f)
+        if ext in (".md", ".json") and stem != "traffic":
+            assert stem in made, f"profiles/{f} is not made by bench.py --ncu all"
