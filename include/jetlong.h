@@ -293,12 +293,22 @@ int jetlong_debug_inject_timeout(int site, long long wait_cycles);
  * NaN stays NaN).  Meant for y <= 2^7, the softmax's range.  d_y, d_out:
  * device float arrays of n elements, n even.
  *
+ * jetlong_debug_rope_keys: the bf16 prefill's key rotation pass on its own --
+ * the range scan of d_k, then d_kl[z][j] = R(j) k[z][j] 2^e and (unless d_kr
+ * is NULL) d_kr[z][j] = R(floor(j / G)) k[z][j] 2^e, as fp16, with 2^e the
+ * power-of-two key scale the prefill would use (e = 13 - floor(log2 max|k|),
+ * clamped to [-100, 100]; 0 for an all-zero or non-finite k).  d_k: bf16
+ * [planes][L][d]; d_kl, d_kr: fp16 of the same shape, 16-byte aligned; *h_exp
+ * (host) receives e, so this call synchronises the stream.
+ *
  * All return JETLONG_OK, JETLONG_ERR_INVALID_ARG or JETLONG_ERR_CUDA;
- * asynchronous on stream. */
+ * asynchronous on stream unless stated. */
 int jetlong_debug_rope_phase(const uint32_t* d_pos, int64_t n, int d, double rope_theta, int accurate,
                              float* d_out, void* stream);
 int jetlong_debug_tile_plan(int P, int C, int w0, int max_kb, int32_t* d_plan, int8_t* d_cls, void* stream);
 int jetlong_debug_ex2(const float* d_y, int64_t n, float* d_out, void* stream);
+int jetlong_debug_rope_keys(const void* d_k, int planes, int L, int d, int G, double rope_theta, void* d_kl,
+                            void* d_kr, int* h_exp, void* stream);
 
 /* Message for the last failing call on this host thread ("" if none). */
 const char* jetlong_last_error(void);

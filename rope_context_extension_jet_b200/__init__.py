@@ -24,7 +24,7 @@ __all__ = [
     "prefill_chunk", "prefill_varlen", "prefill_ie", "prefill_streamed", "decode_workspace_size",
     "decode", "decode_rope_cache", "decode_noalloc", "device_status", "last_error", "launch_count",
     "DECODE_NOALLOC_SCRATCH_BYTES", "selftest_wait_timeout", "debug_inject_timeout",
-    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY", "debug_rope_phase", "debug_tile_plan", "debug_ex2",
+    "INJECT_PREFILL_KEY_TILE", "INJECT_DECODE_COPY", "debug_rope_phase", "debug_tile_plan", "debug_ex2", "debug_rope_keys",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -97,6 +97,8 @@ def load_library(path: str | None = None):
         lib.jetlong_debug_tile_plan.argtypes = [i32, i32, i32, i32, vp, vp, vp]
         lib.jetlong_debug_ex2.restype = i32
         lib.jetlong_debug_ex2.argtypes = [vp, i64, vp, vp]
+        lib.jetlong_debug_rope_keys.restype = i32
+        lib.jetlong_debug_rope_keys.argtypes = [vp, i32, i32, i32, i32, dbl, vp, vp, ctypes.POINTER(ctypes.c_int), vp]
         lib.jetlong_device_status.restype = i32
         lib.jetlong_device_status.argtypes = [vp]
         lib.jetlong_last_error.restype = ctypes.c_char_p
@@ -447,6 +449,26 @@ def debug_ex2(y, stream=None):
     lib = load_library()
     _check(lib.jetlong_debug_ex2(_dev(y, "y"), y.numel(), _dev(out, "out"), _stream(stream)), lib)
     return out
+
+
+def debug_rope_keys(k, G: int, rope_theta: float, remote: bool = True, stream=None):
+    """The bf16 prefill's key rotation pass on its own (test hook
+    jetlong_debug_rope_keys): k, a bf16 CUDA tensor [planes, L, d], rotated to
+    positions j and floor(j / G) times the prefill's key scale 2^e.  Returns
+    (kl, kr or None, e); kl and kr are fp16 tensors of k's shape."""
+    import ctypes as ct
+    import torch
+    if k.dtype != torch.bfloat16 or k.dim() != 3:
+        raise TypeError("k must be a bf16 tensor [planes, L, d]")
+    k = k.contiguous()
+    kl = torch.empty(k.shape, dtype=torch.float16, device=k.device)
+    kr = torch.empty_like(kl) if remote else None
+    ex = ct.c_int(0)
+    lib = load_library()
+    _check(lib.jetlong_debug_rope_keys(_dev(k, "k"), k.shape[0], k.shape[1], k.shape[2], int(G), float(rope_theta),
+                                       _dev(kl, "kl"), _dev(kr, "kr") if remote else None, ct.byref(ex),
+                                       _stream(stream)), lib)
+    return kl, kr, int(ex.value)
 
 
 def device_status(stream=None):

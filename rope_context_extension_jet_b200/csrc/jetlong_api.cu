@@ -680,6 +680,43 @@ int jetlong_debug_ex2(const float* d_y, int64_t n, float* d_out, void* stream)
     return ok();
 }
 
+int jetlong_debug_rope_keys(const void* d_k, int planes, int L, int d, int G, double rope_theta, void* d_kl,
+                            void* d_kr, int* h_exp, void* stream)
+{
+    if (!d_k || !d_kl || !h_exp) return fail(JETLONG_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(d_k) || !aligned16(d_kl) || (d_kr && !aligned16(d_kr)))
+        return fail(JETLONG_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (planes < 1 || L < 1 || (d != 64 && d != 128) || G < 1 || !(rope_theta > 1.0) || !std::isfinite(rope_theta))
+        return fail(JETLONG_ERR_INVALID_ARG, "need planes, L, G >= 1, d in {64, 128}, finite rope_theta > 1");
+    cudaError_t e;
+    uint32_t* slot = next_range_slot(&e);
+    if (!slot) return fail(JETLONG_ERR_CUDA, "range slots: %s", cudaGetErrorString(e));
+    jl::PrefillProblem p{};
+    p.q = d_k; p.k = d_k; p.v = d_k;
+    p.B = planes; p.Hq = 1; p.Hkv = 1; p.L = L; p.d = d;
+    p.P = 0; p.C = L; p.Cst = L; p.Lcap = L;
+    p.G = G;
+    jl::make_rope_turns(&p.turns, d, rope_theta);
+    p.range = slot;
+    int n = 0;
+    e = jl::launch_range_scan(d_k, L, L, planes, d_k, L, L, planes, d, slot, (cudaStream_t)stream, &n);
+    if (e == cudaSuccess) e = jl::launch_rope_keys(p, d_kl, d_kr, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "key rotation launch: %s", cudaGetErrorString(e));
+    uint32_t mag = 0;
+    e = cudaMemcpyAsync(&mag, slot + 1, sizeof mag, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "key scale read: %s", cudaGetErrorString(e));
+    int ex = 0;
+    if (mag != 0u && mag < 0x7f80u) {
+        const int biased = (int)(mag >> 7);
+        ex = 13 - ((biased == 0 ? 1 : biased) - 127);
+        ex = ex < -100 ? -100 : (ex > 100 ? 100 : ex);
+    }
+    *h_exp = ex;
+    return ok();
+}
+
 int jetlong_device_status(void* stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -13,6 +13,12 @@ through a test hook and checked against an independent host computation.
   class against brute-force classification of its causal pairs (local iff
   i - j < w0, Metodologia 1), and the plan's two phases against the sets of key
   blocks holding remote and local pairs.
+* Key rotation pass (jetlong_debug_rope_keys): the bf16 prefill rotates each
+  call's keys once, to j and to floor(j / G), times its power-of-two key scale,
+  into fp16 copies its kernels load.  Checked against the oracle's fp64
+  rotation of the same bf16 keys (row by row at those positions) within fp16
+  rounding plus the fast sine's error, and the scale's exponent against
+  13 - floor(log2 max|k|) from numpy.
 * Softmax exponential on the FMA pipe (jetlong_debug_ex2): 2^y as a quarter of
   the one-CTA prefill's exponentials are formed, against numpy's exp2 in fp64
   over the softmax's range (relative error <= 1e-4, well below the 2^-9 of
@@ -122,3 +128,31 @@ def test_softmax_exp2_on_fma_pipe():
     assert np.all(np.abs(gl[:3]) <= 2.0 ** -125)
     assert np.all(gl[3:7] == 0.0), gl
     assert np.isnan(gl[7])
+
+
+@pytest.mark.parametrize("planes,L,d,G,theta", [(2, 3000, 128, 4, 1e6), (3, 1500, 64, 3, 1e4), (1, 700, 128, 1, 1e6),
+                                               (1, 20000, 128, 5, 1e6)])
+def test_key_rotation_pass_against_oracle(planes, L, d, G, theta):
+    import torch
+    from oracle import rotate, rotate_rows
+    rng = np.random.default_rng(92 + G)
+    k = (rng.standard_normal((planes, L, d)) * 3.0).astype(np.float32)
+    kd = torch.from_numpy(k).to(torch.bfloat16).cuda()
+    kl, kr, e = jl.debug_rope_keys(kd, G, theta, remote=G > 1)
+    jl.device_status()
+    kb = kd.float().cpu().numpy().astype(np.float64)  # the bf16 values the pass reads
+    mx = np.abs(kb).max()
+    assert e == 13 - int(np.floor(np.log2(mx)))
+    scale = 2.0 ** e
+    ref_l = rotate_rows(kb.astype(np.float32), theta) * scale  # bf16 values are exact in fp32
+    checks = [(kl, ref_l, "exact positions")]
+    if G > 1:
+        ref_r = np.stack([np.stack([rotate(kb[z, j], j // G, theta) for j in range(L)]) for z in range(planes)]) * scale
+        checks.append((kr, ref_r, "aliased positions"))
+    # fp16 rounding (half an ulp, 2^-11 relative) plus the fast sine's ~5e-7
+    # absolute error on each factor of a pair (|x| + |y| <= 2 max|k|)
+    for got, ref, what in checks:
+        g = got.double().cpu().numpy()
+        bound = 2.0 ** -11 * np.abs(ref) + 2e-6 * 2 * mx * scale + 1e-7
+        err = np.abs(g - ref) - bound
+        assert err.max() <= 0, f"{what}: worst excess {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
