@@ -152,7 +152,9 @@ int jetlong_prefill_ie(const void* q, const void* k, const void* v, void* out,
                        jetlong_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Prefill from host buffers with the transfers overlapped: the sequence is
- * processed as nchunks chunks of query rows (whole 128-row blocks), and while
+ * processed as min(nchunks, ceil(L / 128)) chunks of query rows (whole 128-row
+ * blocks; the first and the last chunk a quarter of the size of the others,
+ * since nothing overlaps their copy in and out), and while
  * chunk c computes (jetlong_prefill_chunk semantics over the rows uploaded so
  * far) the rows of chunk c + 1 travel host -> device and those of chunk c - 1
  * device -> host, on two copy streams the library keeps per device.

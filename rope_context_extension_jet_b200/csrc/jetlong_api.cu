@@ -4,6 +4,7 @@
 // "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal RoPE"
 // (gist.science/it/paper/2607.07740), Metodologia 1: G = max(1,
 // ceil(L / w_pretrained)) from the current length; f(x) = floor(x / G).
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -444,10 +445,28 @@ int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void*
     cudaError_t e = copy_streams(&h2d, &d2h);
     if (e != cudaSuccess) return fail(JETLONG_ERR_CUDA, "copy streams: %s", cudaGetErrorString(e));
     const size_t row = (size_t)d * (dtype == JETLONG_FP32 ? 4 : 2), pitch = (size_t)L * row;
-    // chunks of whole 128-row query blocks (the last one ragged)
-    int C0 = (L + nchunks - 1) / nchunks;
-    C0 = (C0 + 127) / 128 * 128;
-    const int nch = (L + C0 - 1) / C0;
+    // Chunks of whole 128-row query blocks.  Nothing overlaps the first chunk's
+    // copy in or the last chunk's copy out, and a chunk's compute grows with its
+    // position while its copies do not, so the first and the last chunk get a
+    // quarter of the blocks of each middle chunk.
+    const int nblk = (L + 127) / 128;
+    const int nch = nchunks < nblk ? nchunks : nblk;
+    std::vector<int> first_row(nch + 1, 0);
+    {
+        const int edge = nch > 2 ? std::max(1, (int)std::lround((double)nblk / (2.0 + 4.0 * (nch - 2)))) : 0;
+        const int mid_blocks = nblk - (nch > 2 ? 2 * edge : 0), nmid = nch > 2 ? nch - 2 : nch;
+        int blk = 0;
+        for (int c = 0; c < nch; ++c) {
+            first_row[c] = blk * 128;
+            if (nch > 2 && (c == 0 || c == nch - 1)) {
+                blk += edge;
+            } else {
+                const int m = nch > 2 ? c - 1 : c;  // index among the middle chunks
+                blk += mid_blocks / nmid + (m < mid_blocks % nmid ? 1 : 0);
+            }
+        }
+        first_row[nch] = L;
+    }
     std::vector<cudaEvent_t> ev(2 * nch + 2, nullptr);
     for (auto& x : ev)
         if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) break;
@@ -465,7 +484,7 @@ int jetlong_prefill_streamed(const void* q_host, const void* k_host, const void*
     if ((e = cudaEventRecord(ev[0], cs)) == cudaSuccess && (e = cudaStreamWaitEvent(h2d, ev[0], 0)) == cudaSuccess)
         e = cudaStreamWaitEvent(d2h, ev[0], 0);
     for (int c = 0; c < nch && e == cudaSuccess && st == JETLONG_OK; ++c) {
-        const int P = c * C0, C = L - P < C0 ? L - P : C0;
+        const int P = first_row[c], C = first_row[c + 1] - P;
         // rows [P, P + C) of every plane in; the chunk's prefill (keys [0, P + C),
         // later rows of the device buffers are outside its tensor maps); rows out
         if ((e = cp(q_dev, q_host, P, C, B * Hq, cudaMemcpyHostToDevice, h2d)) != cudaSuccess) break;

@@ -361,7 +361,7 @@ def test_ie_equals_one_pass_at_128k_sampled():
 
 
 # ---------------------------------------------------------------- host buffers, overlapped copies
-@pytest.mark.parametrize("L,nchunks,Hq,Hkv,dtype", [(1000, 3, 4, 1, "bf16"), (777, 16, 4, 2, "bf16"),
+@pytest.mark.parametrize("L,nchunks,Hq,Hkv,dtype", [(1000, 3, 4, 1, "bf16"), (777, 16, 4, 2, "bf16"), (2000, 5, 4, 1, "bf16"),
                                                     (300, 2, 2, 1, "fp32"), (129, 8, 4, 1, "bf16")])
 def test_streamed_prefill_from_host(L, nchunks, Hq, Hkv, dtype):
     import torch
