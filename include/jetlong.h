@@ -90,8 +90,10 @@ int jetlong_position_map(int32_t* d_out, int64_t L, int64_t w_pretrained, void* 
  * G = 1) that the attention kernel loads tile by tile.  They live in a
  * stream-ordered pool the library keeps per device: allocated and freed on
  * `stream` around the kernels, reused by later calls, and reserved until the
- * process exits.  If the pool cannot grow the call returns JETLONG_ERR_CUDA
- * before any launch of the attention kernel.  The chunked, variable-length,
+ * process exits.  The first bf16 prefill call on a device creates the pool:
+ * make it before any stream capture (later calls allocate from the pool in
+ * stream order, which a capture records).  If the pool cannot grow the call
+ * returns JETLONG_ERR_CUDA before any launch of the attention kernel.  The chunked, variable-length,
  * three-pass and streamed calls do the same per launch. */
 int jetlong_prefill(const void* q, const void* k, const void* v, void* out,
                     int B, int Hq, int Hkv, int L, int d,
